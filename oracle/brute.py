@@ -1,0 +1,74 @@
+"""Pure-Python brute force of the GKDT detection head on tiny inputs.
+
+TEST INFRASTRUCTURE ONLY (same import rule as gkd_oracle). A second,
+structurally different restatement used to pin the numpy oracle: nested lists,
+Python floats (IEEE double), one output element at a time, and the upsample as
+a direct 4-tap sum per pixel instead of separable interpolation matrices.
+Sources as in gkd_oracle: GKD_GGUF model card "Model" (Architecture, Prompts,
+Output bullets) and the GKDT summary page's pipeline paragraph.
+"""
+from __future__ import annotations
+
+import math
+
+
+def taps(d: int, n: int, up: int):
+    """The two source indices and weights that output index d reads
+    (half-pixel rule, align_corners=False, borders clamped)."""
+    s = (d + 0.5) / up - 0.5
+    if s < 0.0:
+        s = 0.0
+    i0 = int(s)                     # s >= 0, so int() is floor
+    i1 = i0 + 1 if i0 + 1 < n else n - 1
+    frac = s - i0
+    return (i0, 1.0 - frac), (i1, frac)
+
+
+def up_value(F, h: int, w: int, c: int, Y: int, X: int, up: int) -> float:
+    """Upsampled feature U[Y][X][c] as the 4-tap bilinear sum. F[i][j][c]."""
+    total = 0.0
+    for (iy, wy) in taps(Y, h, up):
+        for (ix, wx) in taps(X, w, up):
+            total += wy * wx * F[iy][ix][c]
+    return total
+
+
+def heat_value(F, h: int, w: int, C: int, kern_row, Y: int, X: int, up: int, rnd=None) -> float:
+    """sum_c kern_row[c] * U[Y][X][c]; `rnd` optionally rounds each U value first."""
+    acc = 0.0
+    for c in range(C):
+        u = up_value(F, h, w, c, Y, X, up)
+        if rnd is not None:
+            u = rnd(u)
+        acc += kern_row[c] * u
+    return acc
+
+
+def pool_row(S, h: int, w: int, C: int, x: float, y: float, sigma: float, stride: float):
+    """Gaussian-weighted mean of the support patches around keypoint (x, y)."""
+    d2 = [[(stride * (j + 0.5) - x) ** 2 + (stride * (i + 0.5) - y) ** 2 for j in range(w)]
+          for i in range(h)]
+    dmin = min(min(r) for r in d2)
+    num = [0.0] * C
+    den = 0.0
+    for i in range(h):
+        for j in range(w):
+            wt = math.exp(-(d2[i][j] - dmin) / (2.0 * sigma * sigma))
+            den += wt
+            for c in range(C):
+                num[c] += wt * S[i][j][c]
+    return [v / den for v in num]
+
+
+def norm_row(row, eps: float = 1e-12):
+    n = math.sqrt(sum(v * v for v in row))
+    n = n if n > eps else eps
+    return [v / n for v in row]
+
+
+def argmax_first(values) -> int:
+    best = 0
+    for p in range(1, len(values)):
+        if values[p] > values[best]:
+            best = p
+    return best

@@ -1,0 +1,53 @@
+"""The seeded input generator: shapes, layouts, determinism, subset stability (CPU)."""
+import numpy as np
+
+from prompt_conditioned_keypoint_b200 import synthetic as S
+
+
+def test_subset_equals_full_batch_slice():
+    full = S.make_config(2, crops=range(0, 6))
+    part = S.make_config(2, crops=[4, 1])
+    np.testing.assert_array_equal(part.feat, full.feat[[4, 1]])
+    np.testing.assert_array_equal(part.rows, full.rows[[4, 1]])
+    np.testing.assert_array_equal(part.mask, full.mask[[4, 1]])
+
+
+def test_config_shapes_and_masks():
+    w2 = S.make_config(2, crops=[0, 1, 2])
+    assert w2.feat.shape == (3, 24, 24, 1024) and w2.feat.dtype == np.float32
+    assert w2.rows.shape == (3, 2, 80, 1024) and w2.mask.shape == (3, 2, 80)
+    for i in range(3):
+        n = int(w2.mask[i, 0].sum())
+        assert 5 <= n <= 80 and np.array_equal(w2.mask[i, 0], w2.mask[i, 1])
+        assert w2.mask[i, 0, :n].all() and not w2.mask[i, 0, n:].any()
+    w3 = S.make_config(3, crops=range(12))
+    assert w3.C == 1280
+    for i in range(12):
+        mod = w3.extra["modality"][i]
+        assert w3.mask[i, 0].any() == (mod in (0, 2)) and w3.mask[i, 1].any() == (mod in (1, 2))
+    w1 = S.make_config(1)
+    assert w1.M == 1 and w1.support.shape == (1, 24, 24, 1024) and int(w1.kmask.sum()) == 17
+    assert np.all((w1.kpts >= 0) & (w1.kpts < 384))
+
+
+def test_config4_is_bf16_and_shared():
+    w4 = S.make_config(4, crops=[0, 5])
+    assert w4.feat.dtype == np.uint16 and w4.Bk == 1 and w4.rows.shape == (1, 2, 80, 1024)
+    assert int(w4.mask.sum()) == 34
+    f = S.bf16_bits_to_f32(w4.feat)
+    assert np.isfinite(f).all() and 0.3 < f.std() < 1.5
+
+
+def test_logical_order_draw_then_nhwc():
+    a = S.make_case(3, 1, 4, 5, 8, 2, 1)
+    g = S._rng(3, S._FEAT, 0)
+    raw = g.standard_normal((8, 4, 5), dtype=np.float32)
+    np.testing.assert_array_equal(a.feat[0], raw.transpose(1, 2, 0))
+
+
+def test_bf16_storage_cast_roundtrip():
+    x = np.array([1.0, 1.00390625, -2.5, 3.0e-3], np.float32)
+    bits = S.to_bf16_bits(x)
+    back = S.bf16_bits_to_f32(bits)
+    assert back[0] == 1.0 and back[2] == -2.5
+    assert np.all(np.abs(back - x) <= np.abs(x) * 2.0 ** -8)
