@@ -1,0 +1,200 @@
+/*
+ * gkd.h - C ABI of libgkd, a B200 (sm_100a) implementation of the
+ * parameter-free detection head of GKDT (General Keypoint Detection
+ * Transformer): prompts become 1x1 convolution kernels that are matched against
+ * dense query features to give keypoint heatmaps, which are decoded to
+ * coordinates.
+ *
+ * Sources for the operations (titles and sections of the pages that define them):
+ *   [CARD]  "Asher-1/GKD_GGUF" model card, section "Model": Architecture bullet
+ *           ("parameter-free detection head (bilinear 4x upsample, L2 kernel
+ *           norm, 1x1 kernel conv, per-row mask fusion over prompts padded to
+ *           80 rows)"), Prompts bullet (Gaussian pooling sigma = 14, "both
+ *           (fused per row)"), Output bullet (peak over a 96x96 grid mapped to
+ *           the ROI's normalized -1..1 space plus a confidence score).
+ *   [SUMM]  "GKDT: General Keypoint Detection Transformer" summary page,
+ *           pipeline paragraph (visual prototypes from Gaussian heatmaps on a
+ *           support image; kernels convolve over the query image's features).
+ *   [NOTES] GKDT reading notes (arxiv-cs-cv-2607-00752), section "Method"
+ *           (visual features aggregated into VKP; normalised convolution).
+ *
+ * Conventions shared by every entry point:
+ *   - Tensor arguments are DEVICE pointers owned by the caller. The library
+ *     never frees them, never keeps them after the call returns, allocates no
+ *     device memory, and never synchronises the stream (except
+ *     gkd_check_device_error). Work is enqueued asynchronously on `stream`
+ *     (a cudaStream_t; NULL means the legacy default stream) on the device
+ *     that owns the first tensor argument.
+ *   - Layouts are dense row-major with the last index contiguous, unless a
+ *     batch-stride argument says otherwise. Strides are in ELEMENTS.
+ *   - Masks are uint8 with 0 (absent) or 1 (present) per entry.
+ *   - Arguments are validated on the host before anything is launched. On any
+ *     violation the call returns a non-zero gkd_status, launches nothing, and
+ *     gkd_last_error() describes the problem. Checks: non-null device pointers,
+ *     positive sizes, dtype support, C % 8 == 0, 16-byte alignment of every
+ *     tensor base pointer and of every batch stride in bytes, size limits
+ *     stated per call.
+ *   - Outputs are fully written (entries of invalid rows get the documented
+ *     fill value) except where a call says a region is left unspecified.
+ *   - Results of kernels with bounded internal waits: if a wait times out the
+ *     kernel records it in a device error word and returns early (outputs are
+ *     then unspecified); gkd_check_device_error() reports it as
+ *     GKD_ERR_TIMEOUT.
+ */
+#ifndef GKD_H_
+#define GKD_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GKD_API __attribute__((visibility("default")))
+#else
+#define GKD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gkd_status {
+  GKD_OK = 0,
+  GKD_ERR_ARG = 1,      /* null / non-device pointer, bad enum, bad flag */
+  GKD_ERR_SHAPE = 2,    /* a size is zero, negative, or beyond a stated limit */
+  GKD_ERR_DTYPE = 3,    /* unsupported dtype or dtype combination */
+  GKD_ERR_ALIGN = 4,    /* a pointer or byte stride is not 16-byte aligned */
+  GKD_ERR_CUDA = 5,     /* a CUDA runtime call failed (launch, attribute, ...) */
+  GKD_ERR_TIMEOUT = 6   /* a kernel's bounded wait ran out (see gkd_check_device_error) */
+} gkd_status;
+
+typedef enum gkd_dtype {
+  GKD_F32 = 0,          /* IEEE binary32 */
+  GKD_BF16 = 1          /* bfloat16 (upper half of binary32), stored as 16-bit words */
+} gkd_dtype;
+
+/*
+ * Step 1: Gaussian prototype pooling of support features ([CARD] Prompts
+ * bullet, "soft-fiber Gaussian pooling, sigma=14"; [SUMM] pipeline paragraph;
+ * [NOTES] Method, support features aggregated into visual prototypes).
+ *
+ *   proto[b,k,:] = sum_ij w_ij * support[b,i,j,:] / sum_ij w_ij,
+ *   w_ij = exp(-((X_j - x)^2 + (Y_i - y)^2) / (2 sigma^2)),
+ *   X_j = stride_px * (j + 0.5), Y_i = stride_px * (i + 0.5),
+ * for keypoints with kmask[b,k] != 0; rows of absent keypoints are set to 0.
+ * The weights are evaluated over the whole h x w grid (no truncation).
+ *
+ *   support  [B][h][w][C] (sdt = GKD_F32 only; GKD_BF16 returns GKD_ERR_DTYPE)
+ *   kpts     [B][K][2] fp32, (x, y) in ROI pixels of the support image
+ *   kmask    [B][K] uint8
+ *   proto    fp32; crop b's rows start at proto + b * proto_batch_stride and are
+ *            [K][C] contiguous (proto_batch_stride >= K * C; pass 2*K*C to
+ *            write straight into modality 0 of a [B][2][K][C] row tensor).
+ * Limits: 1 <= K <= 128, 1 <= h, w <= 256, B <= 65535,
+ *         4 * K * (2 + h + w) <= 200 KiB, sigma_px > 0, stride_px > 0.
+ */
+GKD_API gkd_status gkd_pool_prototypes(const void* support, gkd_dtype sdt, int B, int h, int w, int C,
+                               const float* kpts, const uint8_t* kmask, int K, float sigma_px,
+                               float stride_px, float* proto, long long proto_batch_stride,
+                               void* stream);
+
+/*
+ * Step 2: L2 normalisation of prompt rows ([CARD] Architecture bullet,
+ * "L2 kernel norm ... prompts padded to 80 rows"; [NOTES] Method, normalised
+ * convolution).
+ *
+ *   out[r,:] = rows[r,:] / max(||rows[r,:]||_2, eps)  where mask[r] != 0,
+ *   out[r,:] = 0                                       where mask[r] == 0,
+ * over the Bk*M*K rows of rows [Bk][M][K][C] (fp32) with mask [Bk][M][K].
+ * Sum of squares in fp32, IEEE square root and division. out_dt = GKD_BF16
+ * rounds the fp32 quotient to bf16 (nearest, ties to even).
+ *   out  [Bk][M][K][C], fp32 or bf16 per out_dt.
+ * Limits: 1 <= M <= 2, 1 <= K <= 128, eps > 0, Bk*M*K < 2^31.
+ */
+GKD_API gkd_status gkd_norm_kernels(const float* rows, const uint8_t* mask, int Bk, int M, int K, int C, float eps,
+                            gkd_dtype out_dt, void* out, void* stream);
+
+/*
+ * Steps 3 + 4: bilinear 4x upsample of the query features (align_corners =
+ * False, half-pixel source coordinate s = max((d + 0.5)/4 - 0.5, 0), upper
+ * neighbour clamped to the last row/column) fused into the 1x1 dynamic-kernel
+ * contraction ([CARD] Architecture bullet, "bilinear 4x upsample, ... 1x1
+ * kernel conv"; [CARD] Output bullet, 96x96 grid; [SUMM] "kernels convolve over
+ * the query image's features"):
+ *
+ *   heat[b,m,k,Y,X] = sum_c kern[b,m,k,c] * U[b,Y,X,c]   for mask[b,m,k] != 0.
+ *
+ *   feat    [B][h][w][C], fdt = GKD_F32 or GKD_BF16
+ *   kern    crop b's rows at kern + b * kern_batch_stride, [M][K][C];
+ *           kern_batch_stride = 0 shares one prompt set across all crops.
+ *           kdt = GKD_BF16: tensor-core path. U is formed in fp32 and rounded
+ *             to bf16 (nearest even); products are summed in fp32.
+ *           kdt = GKD_F32 (requires fdt = GKD_F32): fp32 path, U and the sum in
+ *             fp32.
+ *   mask    crop b's [M][K] at mask + b * mask_batch_stride (0 = shared)
+ *   heat    [B][M][K][4h][4w] fp32. Rows with mask == 0 are NOT written
+ *           (left unspecified).
+ * Limits: up == 4, 1 <= M <= 2, 1 <= K <= 128, M * ceil8(K) <= 160 on the bf16
+ *         path, 1 <= h, w <= 256, B <= 65535, C % 8 == 0.
+ */
+GKD_API gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up,
+                       const void* kern, gkd_dtype kdt, long long kern_batch_stride,
+                       const uint8_t* mask, long long mask_batch_stride, int M, int K,
+                       float* heat, void* stream);
+
+/*
+ * Step 5: per-row masked fusion across modalities and peak decode ([CARD]
+ * Architecture bullet, "per-row mask fusion"; Prompts bullet, "both (fused
+ * per row)"; Output bullet, peak -> ROI -1..1 + confidence score).
+ *
+ * For each (b, k): cnt = number of modalities m with mask[b,m,k] != 0;
+ *   fused = heat[b,m,k] for the one present modality, or
+ *           (heat[b,0,k] + heat[b,1,k]) * 0.5 in fp32 when both are;
+ *   idx   = first (lowest row-major index Y*W + X) maximal pixel of fused;
+ *   score = fused[idx];
+ *   xy    = ((2 X + 1 - W) / W, (2 Y + 1 - H) / H), one IEEE fp32 division each
+ *           (= 2 (X + 0.5)/W - 1, correctly rounded);
+ *   valid = 1.
+ * Rows with cnt == 0: idx = -1, xy = (0, 0), score = 0, valid = 0, fused row 0.
+ *
+ *   heat   [B][M][K][H][W] fp32 (rows with mask 0 are not read)
+ *   mask   crop b's [M][K] at mask + b * mask_batch_stride (0 = shared)
+ *   fused  optional [B][K][H][W] fp32 (NULL: not written)
+ *   xy [B][K][2] fp32, score [B][K] fp32, idx [B][K] int32, valid [B][K] uint8
+ * Limits: 1 <= M <= 2, 1 <= K <= 65535, H * W % 4 == 0, H * W < 2^31, B <= 65535.
+ */
+GKD_API gkd_status gkd_fuse_decode(const float* heat, const uint8_t* mask, long long mask_batch_stride, int B, int M,
+                           int K, int H, int W, float* fused, float* xy, float* score, int32_t* idx,
+                           uint8_t* valid, void* stream);
+
+/* Message for the last non-OK status returned on the calling thread ("" if none). */
+GKD_API const char* gkd_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's error
+ * word. Returns GKD_ERR_TIMEOUT if a kernel's bounded wait ran out since the
+ * last check, GKD_ERR_CUDA if the stream reports a CUDA error, else GKD_OK.
+ */
+GKD_API gkd_status gkd_check_device_error(void* stream);
+
+/*
+ * Upper bound, in milliseconds, on any single internal wait of the tensor-core
+ * heatmap kernel (default 2000). Process-wide; applies to later launches.
+ * Returns GKD_ERR_ARG for 0.
+ */
+GKD_API gkd_status gkd_set_wait_timeout_ms(unsigned int ms);
+
+/*
+ * Test hook: bit 0 makes the next gkd_heatmap launch on the bf16 path withhold
+ * its upsample producers' first hand-off to the MMA warp, so the MMA warp's
+ * bounded wait runs out and the kernel takes its timeout exit. The flags are
+ * consumed (reset to 0) by that launch. Returns GKD_ERR_ARG for unknown bits.
+ */
+GKD_API gkd_status gkd_debug_set_flags(unsigned int flags);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+GKD_API int gkd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GKD_H_ */

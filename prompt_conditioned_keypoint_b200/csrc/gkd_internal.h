@@ -1,0 +1,63 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+// Every launcher assumes its arguments were validated by the caller and only
+// enqueues work on `stream`; it returns the CUDA launch status.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace gkd {
+
+// Device error word bits (written by kernels, read by gkd_check_device_error).
+enum : unsigned {
+  kErrTimeout = 1u << 0,   // a bounded wait ran out
+  kErrBounds = 1u << 1,    // a debug-build bounds check fired
+};
+
+// Test hooks for the forced-timeout path (host-set, consumed by the next launch).
+enum : unsigned {
+  kDbgSkipProducerArrive = 1u << 0,   // upsample producers never signal their first stage
+};
+
+cudaError_t launch_pool(const float* support, int B, int h, int w, int C, const float* kpts,
+                        const uint8_t* kmask, int K, float sigma, float stride, float* proto,
+                        long long proto_batch_stride, cudaStream_t stream);
+
+cudaError_t launch_norm(const float* rows, const uint8_t* mask, long long nrows, int C, float eps,
+                        bool out_bf16, void* out, cudaStream_t stream);
+
+cudaError_t launch_fuse_decode(const float* heat, const uint8_t* mask, long long mask_batch_stride,
+                               int B, int M, int K, int H, int W, float* fused, float* xy, float* score,
+                               int32_t* idx, uint8_t* valid, cudaStream_t stream);
+
+cudaError_t launch_heatmap_f32(const float* feat, int B, int h, int w, int C, const float* kern,
+                               long long kern_batch_stride, const uint8_t* mask, long long mask_batch_stride,
+                               int M, int K, float* heat, cudaStream_t stream);
+
+struct HeatmapTcArgs {
+  CUtensorMap tmap_feat;     // feature slabs  {C, w, h, B}
+  CUtensorMap tmap_kern8;    // kernel rows, 8-row boxes  {C, K, M, Bk}
+  CUtensorMap tmap_kern32;   // kernel rows, 32-row boxes
+  const uint8_t* mask;
+  long long mask_batch_stride;
+  float* heat;
+  int B, h, w, C, M, K;
+  int feat_bf16;
+  int kern_shared;           // kernels shared by all crops (batch stride 0)
+  unsigned* err;             // device error word
+  unsigned long long wait_limit_ns;
+  unsigned debug_flags;
+};
+
+// Encodes the tensor maps and launches the persistent tcgen05 kernel.
+cudaError_t launch_heatmap_tc(HeatmapTcArgs& a, const void* feat, const void* kern,
+                              long long kern_batch_stride, int num_sms, cudaStream_t stream,
+                              const char** why);
+
+// cuTensorMapEncodeTiled resolved through the runtime's driver entry point.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+}  // namespace gkd

@@ -1,0 +1,185 @@
+"""The detection head as one call sequence over libgkd (device memory via torch).
+
+`GkdHead` owns the device buffers of one batch shape and enqueues the head's
+steps through the C ABI on a stream:
+
+  [gkd_pool_prototypes]   visual rows from support maps (when keypoints are given)
+  gkd_norm_kernels        L2-normalised rows (bf16 or fp32 operands)
+  gkd_heatmap             fused 4x upsample + 1x1 contraction
+  gkd_fuse_decode         per-row modality fusion + peak decode
+
+torch only allocates memory, owns streams and copies host buffers; every step
+of the head runs in libgkd's kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import binding as gk
+
+DTYPE_CODE = {"f32": gk.GKD_F32, "bf16": gk.GKD_BF16}
+
+
+@dataclass(frozen=True)
+class HeadShape:
+    B: int
+    h: int
+    w: int
+    C: int
+    K: int
+    M: int
+    feat_dtype: str = "f32"       # "f32" | "bf16"
+    kern_dtype: str = "bf16"      # operand type of the contraction: "f32" | "bf16"
+    shared: bool = False          # one prompt set for all crops
+    pooled: bool = False          # modality 0 rows come from Gaussian pooling
+    sigma: float = 14.0
+    stride: float = 16.0
+    up: int = 4
+
+    @property
+    def Bk(self) -> int:
+        return 1 if self.shared else self.B
+
+    @property
+    def H(self) -> int:
+        return self.up * self.h
+
+    @property
+    def W(self) -> int:
+        return self.up * self.w
+
+    @staticmethod
+    def of(wl) -> "HeadShape":
+        return HeadShape(wl.B, wl.h, wl.w, wl.C, wl.K, wl.M, wl.feat_dtype, wl.kern_dtype, wl.Bk == 1,
+                         wl.support is not None, float(wl.sigma), float(wl.stride), wl.up)
+
+    def launches_per_step(self) -> int:
+        return 3 + (1 if self.pooled else 0)
+
+
+class GkdHead:
+    def __init__(self, shape: HeadShape, device, with_fused: bool = False):
+        s = self.shape = shape
+        d = self.device = torch.device(device)
+        fdt = torch.float32 if s.feat_dtype == "f32" else torch.int16
+        self.feat = torch.empty((s.B, s.h, s.w, s.C), dtype=fdt, device=d)
+        self.rows = torch.zeros((s.Bk, s.M, s.K, s.C), dtype=torch.float32, device=d)
+        self.mask = torch.zeros((s.Bk, s.M, s.K), dtype=torch.uint8, device=d)
+        kdt = torch.float32 if s.kern_dtype == "f32" else torch.int16
+        self.khat = torch.empty((s.Bk, s.M, s.K, s.C), dtype=kdt, device=d)
+        if s.pooled:
+            self.support = torch.empty((s.B, s.h, s.w, s.C), dtype=torch.float32, device=d)
+            self.kpts = torch.empty((s.B, s.K, 2), dtype=torch.float32, device=d)
+            self.kmask = torch.empty((s.B, s.K), dtype=torch.uint8, device=d)
+        self.heat = torch.empty((s.B, s.M, s.K, s.H, s.W), dtype=torch.float32, device=d)
+        self.fused = torch.empty((s.B, s.K, s.H, s.W), dtype=torch.float32, device=d) if with_fused else None
+        self.xy = torch.empty((s.B, s.K, 2), dtype=torch.float32, device=d)
+        self.score = torch.empty((s.B, s.K), dtype=torch.float32, device=d)
+        self.idx = torch.empty((s.B, s.K), dtype=torch.int32, device=d)
+        self.valid = torch.empty((s.B, s.K), dtype=torch.uint8, device=d)
+
+    # ------------------------------------------------------------------ inputs
+    def host_inputs(self, wl, pin: bool = True) -> dict:
+        """Host tensors (pinned) of a synthetic workload, in this head's layouts."""
+        s = self.shape
+        feat = wl.feat.view(np.int16) if s.feat_dtype == "bf16" else wl.feat
+        out = {"feat": torch.from_numpy(np.ascontiguousarray(feat)), "mask": torch.from_numpy(wl.mask)}
+        if s.pooled:
+            out["support"] = torch.from_numpy(wl.support)
+            out["kpts"] = torch.from_numpy(wl.kpts)
+            out["kmask"] = torch.from_numpy(wl.kmask)
+            if s.M == 2:
+                out["text_rows"] = torch.from_numpy(np.ascontiguousarray(wl.rows[:, 1]))
+        else:
+            out["rows"] = torch.from_numpy(wl.rows)
+        if pin:
+            out = {k: v.pin_memory() for k, v in out.items()}
+        return out
+
+    def upload(self, host: dict, stream=None):
+        """Copy host inputs into the device buffers on `stream` (asynchronously when pinned)."""
+        st = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(st):
+            self.feat.copy_(host["feat"], non_blocking=True)
+            self.mask.copy_(host["mask"], non_blocking=True)
+            if self.shape.pooled:
+                self.support.copy_(host["support"], non_blocking=True)
+                self.kpts.copy_(host["kpts"], non_blocking=True)
+                self.kmask.copy_(host["kmask"], non_blocking=True)
+                if "text_rows" in host:
+                    self.rows[:, 1].copy_(host["text_rows"], non_blocking=True)
+            else:
+                self.rows.copy_(host["rows"], non_blocking=True)
+
+    def host_input_bytes(self, host: dict) -> int:
+        return sum(v.numel() * v.element_size() for v in host.values())
+
+    # ------------------------------------------------------------------ steps
+    def pool(self, stream=None):
+        s = self.shape
+        gk.gkd_pool_prototypes(self.support, gk.GKD_F32, s.B, s.h, s.w, s.C, self.kpts, self.kmask, s.K,
+                               s.sigma, s.stride, self.rows, s.M * s.K * s.C, stream)
+
+    def norm(self, stream=None):
+        s = self.shape
+        gk.gkd_norm_kernels(self.rows, self.mask, s.Bk, s.M, s.K, s.C, 1e-12, DTYPE_CODE[s.kern_dtype],
+                            self.khat, stream)
+
+    def heatmap(self, stream=None):
+        s = self.shape
+        kbs = 0 if s.shared else s.M * s.K * s.C
+        mbs = 0 if s.shared else s.M * s.K
+        gk.gkd_heatmap(self.feat, DTYPE_CODE[s.feat_dtype], s.B, s.h, s.w, s.C, s.up, self.khat,
+                       DTYPE_CODE[s.kern_dtype], kbs, self.mask, mbs, s.M, s.K, self.heat, stream)
+
+    def fuse_decode(self, stream=None):
+        s = self.shape
+        mbs = 0 if s.shared else s.M * s.K
+        gk.gkd_fuse_decode(self.heat, self.mask, mbs, s.B, s.M, s.K, s.H, s.W, self.fused, self.xy, self.score,
+                           self.idx, self.valid, stream)
+
+    def forward(self, stream=None, heatmap_events=None):
+        """Enqueue the whole head. `heatmap_events` = (start, end) CUDA events
+        recorded around the heatmap launch on the same stream."""
+        st = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if self.shape.pooled:
+            self.pool(st)
+        self.norm(st)
+        if heatmap_events is not None:
+            heatmap_events[0].record(st)
+        self.heatmap(st)
+        if heatmap_events is not None:
+            heatmap_events[1].record(st)
+        self.fuse_decode(st)
+
+    def outputs_to_host(self, dst: dict | None = None, stream=None) -> dict:
+        st = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if dst is None:
+            dst = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                   for k, v in (("xy", self.xy), ("score", self.score), ("idx", self.idx), ("valid", self.valid))}
+        with torch.cuda.stream(st):
+            dst["xy"].copy_(self.xy, non_blocking=True)
+            dst["score"].copy_(self.score, non_blocking=True)
+            dst["idx"].copy_(self.idx, non_blocking=True)
+            dst["valid"].copy_(self.valid, non_blocking=True)
+        return dst
+
+    def output_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.xy, self.score, self.idx, self.valid))
+
+    def run_host(self, host: dict, out: dict | None = None, stream=None) -> dict:
+        """End to end through the public API: host inputs in, decoded keypoints out."""
+        st = stream if stream is not None else torch.cuda.current_stream(self.device)
+        self.upload(host, st)
+        self.forward(st)
+        return self.outputs_to_host(out, st)
+
+    def algorithmic_heatmap_flops(self, mask: np.ndarray) -> float:
+        """2 * R * C * P summed over crops, R = valid rows of each crop."""
+        s = self.shape
+        rows = mask.reshape(mask.shape[0], -1).sum(axis=1).astype(np.float64)
+        total_rows = rows[0] * s.B if s.shared else rows.sum()
+        return 2.0 * total_rows * s.C * s.H * s.W

@@ -1,0 +1,330 @@
+"""GPU parity: each libgkd call against the CPU oracle on the same seeded inputs.
+
+Small shapes span several tiles, ragged channel chunks, ragged pixel tiles and
+the degenerate cases; the five workloads run at full size with sampled crops
+compared against the oracle one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import (BF16_TOL, F32_TOL, assert_rows_close, bf16_dev, check_decode_against_margin, dev,
+                         to_dev, valid_heat_rows)
+from oracle import gkd_oracle as O
+from prompt_conditioned_keypoint_b200 import binding as gk
+from prompt_conditioned_keypoint_b200 import synthetic as S
+from prompt_conditioned_keypoint_b200.head import GkdHead, HeadShape
+
+pytestmark = pytest.mark.gpu
+
+
+def sync_check():
+    torch.cuda.synchronize()
+    gk.gkd_check_device_error()
+
+
+# ----------------------------------------------------------------------------- a2
+@pytest.mark.parametrize("out_dt", ["f32", "bf16"])
+def test_norm_parity(out_dt):
+    rng = np.random.default_rng(5)
+    rows = rng.standard_normal((3, 2, 80, 1280)).astype(np.float32)
+    rows[0, 1, 4] = 0.0                       # zero row, valid: stays 0 (0 / eps)
+    rows[1, 0, 7] *= 1e-12                    # tiny norm (squares stay normal fp32)
+    mask = (rng.random((3, 2, 80)) < 0.7).astype(np.uint8)
+    mask[0, 1, 4] = 1
+    out = torch.empty((3, 2, 80, 1280), dtype=torch.float32 if out_dt == "f32" else torch.int16, device=dev())
+    out.fill_(7)
+    gk.gkd_norm_kernels(to_dev(rows), to_dev(mask), 3, 2, 80, 1280, 1e-12,
+                        gk.GKD_F32 if out_dt == "f32" else gk.GKD_BF16, out)
+    sync_check()
+    ref = O.norm_rows(rows.astype(np.float64), mask)
+    if out_dt == "f32":
+        got = out.cpu().numpy().astype(np.float64)
+        assert_rows_close(got.reshape(-1, 1280), ref.reshape(-1, 1280) + 0.0, F32_TOL, "norm f32")
+        assert np.all(got[mask == 0] == 0)
+    else:
+        got = O.bf16_decode(out.cpu().numpy().view(np.uint16))
+        want = O.bf16_round(ref)
+        diff = got != want
+        # fp32 quotient then bf16 vs direct fp64 -> bf16: rare one-ulp double-rounding flips only
+        assert diff.mean() < 1e-3, diff.mean()
+        ulp = np.abs(want[diff]) * 2.0 ** -7
+        assert np.all(np.abs(got[diff] - want[diff]) <= ulp + 1e-45)
+        assert np.all(got[mask == 0] == 0)
+
+
+# ----------------------------------------------------------------------------- a1
+@pytest.mark.parametrize("case", [
+    dict(B=2, h=24, w=24, C=256, K=80, sigma=14.0, stride=16.0),
+    dict(B=2, h=48, w=48, C=128, K=80, sigma=28.0, stride=16.0),
+    dict(B=3, h=5, w=7, C=40, K=9, sigma=9.0, stride=16.0),
+    dict(B=1, h=1, w=1, C=8, K=1, sigma=14.0, stride=16.0),
+])
+def test_pool_parity(case):
+    support, kpts, kmask = S.make_pool_case(11, case["B"], case["h"], case["w"], case["C"], case["K"],
+                                            sigma=case["sigma"], stride=case["stride"])
+    kmask[0, 0] = 1
+    B, h, w, C, K = case["B"], case["h"], case["w"], case["C"], case["K"]
+    proto = torch.full((B, K, C), 5.0, device=dev())
+    gk.gkd_pool_prototypes(to_dev(support), gk.GKD_F32, B, h, w, C, to_dev(kpts), to_dev(kmask), K,
+                           case["sigma"], case["stride"], proto, K * C)
+    sync_check()
+    got = proto.cpu().numpy()
+    ref = O.pool_prototypes(support, kpts, kmask, case["sigma"], case["stride"])
+    sel = kmask.reshape(-1) == 1
+    assert_rows_close(got.reshape(-1, C)[sel], ref.reshape(-1, C)[sel], F32_TOL, "pool")
+    assert np.all(got.reshape(-1, C)[~sel] == 0)
+
+
+def test_pool_strided_output_and_small_sigma():
+    B, h, w, C, K = 2, 24, 24, 64, 4
+    support, _, _ = S.make_pool_case(3, B, h, w, C, K)
+    kpts = np.array([[[16 * 3 + 8, 16 * 17 + 8]] * K] * B, np.float32)
+    kmask = np.ones((B, K), np.uint8)
+    rows = torch.full((B, 2, K, C), -1.0, device=dev())
+    gk.gkd_pool_prototypes(to_dev(support), gk.GKD_F32, B, h, w, C, to_dev(kpts), to_dev(kmask), K, 0.1, 16.0,
+                           rows, 2 * K * C)
+    sync_check()
+    got = rows.cpu().numpy()
+    for b in range(B):
+        np.testing.assert_allclose(got[b, 0], np.broadcast_to(support[b, 17, 3], (K, C)), rtol=0, atol=0)
+    assert np.all(got[:, 1] == -1.0)          # modality 1 untouched by the strided write
+
+
+# ----------------------------------------------------------------------------- a3 + a4
+def run_heatmap(wl, kern_bits_or_f32):
+    s = wl
+    Bk = s.Bk
+    feat = bf16_dev(s.feat) if s.feat_dtype == "bf16" else to_dev(s.feat)
+    kern = bf16_dev(kern_bits_or_f32) if s.kern_dtype == "bf16" else to_dev(kern_bits_or_f32)
+    heat = torch.full((s.B, s.M, s.K, 4 * s.h, 4 * s.w), float("nan"), device=dev())
+    kbs = 0 if Bk == 1 else s.M * s.K * s.C
+    mbs = 0 if Bk == 1 else s.M * s.K
+    gk.gkd_heatmap(feat, gk.GKD_BF16 if s.feat_dtype == "bf16" else gk.GKD_F32, s.B, s.h, s.w, s.C, 4, kern,
+                   gk.GKD_BF16 if s.kern_dtype == "bf16" else gk.GKD_F32, kbs, to_dev(s.mask), mbs, s.M, s.K, heat)
+    sync_check()
+    return heat.cpu().numpy()
+
+
+def feat64(wl, crops=None):
+    f = wl.feat if crops is None else wl.feat[crops]
+    return O.bf16_decode(f) if wl.feat_dtype == "bf16" else f.astype(np.float64)
+
+
+HEAT_CASES = [
+    dict(seed=21, B=2, h=24, w=24, C=256, K=80, M=2, feat_dtype="f32", valid="prefix"),
+    dict(seed=22, B=3, h=5, w=7, C=200, K=13, M=2, feat_dtype="f32", valid="random"),
+    dict(seed=23, B=2, h=24, w=24, C=136, K=17, M=2, feat_dtype="bf16", valid="all", shared=True),
+    dict(seed=24, B=1, h=1, w=1, C=8, K=1, M=1, feat_dtype="f32", valid="all"),
+    dict(seed=25, B=2, h=12, w=12, C=128, K=80, M=2, feat_dtype="f32", valid="all"),
+    dict(seed=26, B=2, h=3, w=9, C=64, K=128, M=1, feat_dtype="bf16", valid="random"),
+    dict(seed=27, B=40, h=8, w=8, C=64, K=20, M=2, feat_dtype="f32", valid="random"),
+    dict(seed=28, B=1, h=48, w=48, C=72, K=5, M=2, feat_dtype="f32", valid="prefix"),
+]
+
+
+@pytest.mark.parametrize("case", HEAT_CASES, ids=lambda c: f"s{c['seed']}")
+def test_heatmap_bf16_parity(case):
+    c = dict(case)
+    wl = S.make_case(c.pop("seed"), c.pop("B"), c.pop("h"), c.pop("w"), c.pop("C"), c.pop("K"), c.pop("M"),
+                     kern_dtype="bf16", **c)
+    if wl.B == 40:
+        wl.mask[5] = 0                         # crops with no valid row at all
+        wl.mask[6] = 0
+    kern = S.random_bf16_rows(case["seed"], (wl.Bk, wl.M, wl.K, wl.C), 1.0 / np.sqrt(wl.C))
+    got = run_heatmap(wl, kern)
+    ref = O.heatmaps(feat64(wl), O.bf16_decode(kern), wl.mask, 4, "bf16")
+    g, sel = valid_heat_rows(got, wl.mask)
+    r, _ = valid_heat_rows(ref, wl.mask)
+    if sel:
+        assert_rows_close(g, r, BF16_TOL, "heatmap bf16")
+        # matched rounding points: nearly every element agrees to fp32 accuracy; the rest are
+        # single bf16 double-rounding flips of U (fp32 lerp then bf16, versus fp64 then bf16)
+        rel = np.abs(g - r) / np.abs(r).max(axis=(1, 2), keepdims=True)
+        assert (rel > 1e-5).mean() < 0.1, (rel > 1e-5).mean()
+
+
+@pytest.mark.parametrize("case", [
+    dict(seed=31, B=1, h=24, w=24, C=1024, K=80, M=1, valid="prefix"),
+    dict(seed=32, B=2, h=5, w=7, C=200, K=13, M=2, valid="random"),
+    dict(seed=33, B=2, h=24, w=24, C=96, K=17, M=2, valid="all", shared=True),
+], ids=lambda c: f"s{c['seed']}")
+def test_heatmap_f32_parity(case):
+    c = dict(case)
+    wl = S.make_case(c.pop("seed"), c.pop("B"), c.pop("h"), c.pop("w"), c.pop("C"), c.pop("K"), c.pop("M"),
+                     kern_dtype="f32", **c)
+    rng = np.random.default_rng(case["seed"])
+    kern = (rng.standard_normal((wl.Bk, wl.M, wl.K, wl.C)) / np.sqrt(wl.C)).astype(np.float32)
+    got = run_heatmap(wl, kern)
+    ref = O.heatmaps(feat64(wl), kern.astype(np.float64), wl.mask, 4, "f32")
+    g, sel = valid_heat_rows(got, wl.mask)
+    r, _ = valid_heat_rows(ref, wl.mask)
+    assert_rows_close(g, r, F32_TOL, "heatmap f32")
+
+
+def test_heatmap_onehot_and_constant_closed_forms():
+    # one-hot channel at an interior cell matched with the same unit kernel: peak 49/64 exactly
+    B, h, w, C, K = 1, 24, 24, 64, 2
+    feat = np.zeros((B, h, w, C), np.float32)
+    feat[0, 5, 7, 3] = 1.0
+    feat[0, :, :, 10] = 3.25                   # constant channel
+    kern = np.zeros((1, 1, K, C), np.float32)
+    kern[0, 0, 0, 3] = 1.0
+    kern[0, 0, 1, 10] = 1.0
+    bits = S.to_bf16_bits(kern)
+    wl = S.Workload("onehot", B, h, w, C, K, 1, 4, feat, "f32", None, np.ones((1, 1, K), np.uint8), 1, "bf16")
+    got = run_heatmap(wl, bits)
+    assert got[0, 0, 0].max() == 0.765625
+    ys, xs = np.nonzero(got[0, 0, 0] == 0.765625)
+    assert set(ys) == {21, 22} and set(xs) == {29, 30}
+    assert np.all(got[0, 0, 1] == 3.25)
+
+
+# ----------------------------------------------------------------------------- a5 + a6
+@pytest.mark.parametrize("M", [1, 2])
+def test_fuse_decode_bit_exact(M):
+    B, K, H, W = 3, 9, 96, 96
+    heat = S.random_heatmaps(41 + M, B, M, K, H, W)
+    rng = np.random.default_rng(M)
+    mask = (rng.random((B, M, K)) < 0.7).astype(np.uint8)
+    mask[0, :, 0] = 0                          # a row with no modality present
+    mask[1, :, 1] = 1
+    fused = torch.full((B, K, H, W), 9.0, device=dev())
+    xy = torch.full((B, K, 2), 9.0, device=dev())
+    score = torch.full((B, K), 9.0, device=dev())
+    idx = torch.full((B, K), 9, dtype=torch.int32, device=dev())
+    valid = torch.full((B, K), 9, dtype=torch.uint8, device=dev())
+    gk.gkd_fuse_decode(to_dev(heat), to_dev(mask), M * K, B, M, K, H, W, fused, xy, score, idx, valid)
+    sync_check()
+    rf, ri, rxy, rs, rv = O.fuse_decode(heat, mask)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ri)
+    np.testing.assert_array_equal(valid.cpu().numpy(), rv)
+    np.testing.assert_array_equal(score.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    np.testing.assert_array_equal(xy.cpu().numpy().view(np.uint32), rxy.view(np.uint32))
+    np.testing.assert_array_equal(fused.cpu().numpy().view(np.uint32), rf.view(np.uint32))
+
+
+def test_fuse_decode_shared_mask_and_tiny_grid():
+    B, M, K, H, W = 2, 2, 3, 4, 4
+    heat = S.random_heatmaps(7, B, M, K, H, W)
+    mask = np.array([[[1, 0, 1], [1, 1, 0]]], np.uint8)
+    outs = [torch.empty((B, K, 2), device=dev()), torch.empty((B, K), device=dev()),
+            torch.empty((B, K), dtype=torch.int32, device=dev()), torch.empty((B, K), dtype=torch.uint8, device=dev())]
+    gk.gkd_fuse_decode(to_dev(heat), to_dev(mask), 0, B, M, K, H, W, None, *outs)
+    sync_check()
+    _, ri, rxy, rs, rv = O.fuse_decode(heat, mask)
+    np.testing.assert_array_equal(outs[2].cpu().numpy(), ri)
+    np.testing.assert_array_equal(outs[0].cpu().numpy().view(np.uint32), rxy.view(np.uint32))
+    np.testing.assert_array_equal(outs[1].cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    np.testing.assert_array_equal(outs[3].cpu().numpy(), rv)
+
+
+# ----------------------------------------------------------------------------- the five workloads
+_RUNS = {}
+
+
+def run_config(cfg):
+    """Full-size workload through the whole head on the GPU (cached per module)."""
+    if cfg not in _RUNS:
+        _RUNS.clear()
+        torch.cuda.empty_cache()
+        wl = S.make_config(cfg)
+        head = GkdHead(HeadShape.of(wl), dev(), with_fused=False)
+        head.upload(head.host_inputs(wl, pin=False))
+        head.forward()
+        sync_check()
+        _RUNS[cfg] = (wl, head)
+    return _RUNS[cfg]
+
+
+def oracle_rows(wl, crops):
+    """Raw (pre-normalisation) rows of the selected crops, pooling first where the workload pools."""
+    if wl.support is None:
+        return wl.rows.astype(np.float64) if wl.Bk == 1 else wl.rows[crops].astype(np.float64)
+    proto = O.pool_prototypes(wl.support[crops], wl.kpts[crops], wl.kmask[crops], wl.sigma, wl.stride)
+    rows = np.zeros((len(crops), wl.M, wl.K, wl.C))
+    rows[:, 0] = proto
+    if wl.M == 2:
+        rows[:, 1] = wl.rows[crops, 1]
+    return rows
+
+
+@pytest.mark.parametrize("cfg,crops", [(1, [0]), (2, [0, 17, 63]), (3, [0, 101, 255]), (4, [0, 511, 1023]),
+                                       (5, [0, 31])], ids=["w1", "w2", "w3", "w4", "w5"])
+def test_workload_parity(cfg, crops):
+    wl, head = run_config(cfg)
+    operand = wl.kern_dtype
+    tol = F32_TOL if operand == "f32" else BF16_TOL
+    rows = oracle_rows(wl, crops)
+    mask = wl.mask if wl.Bk == 1 else wl.mask[crops]
+    f64 = feat64(wl, crops)
+    heat_ref, (fused_ref, _, _, _, valid_ref) = O.head(f64, rows, mask, operand=operand)
+    heat = head.heat[crops].cpu().numpy()
+    g, sel = valid_heat_rows(heat, mask)
+    r, _ = valid_heat_rows(heat_ref, mask)
+    worst = assert_rows_close(g, r, tol, f"workload {cfg} heatmaps")
+    print(f"workload {cfg}: worst heat row error {worst:.2e} (tol {tol:.0e})")
+    idx = head.idx.cpu().numpy()[crops]
+    valid = head.valid.cpu().numpy()[crops]
+    checked, skipped = check_decode_against_margin(fused_ref, valid_ref, idx, valid, tol)
+    assert checked > 0
+    print(f"workload {cfg}: argmax bit-exact on {checked} rows, {skipped} near-ties skipped")
+    # xy follows idx by the fixed formula
+    xy = head.xy.cpu().numpy()[crops]
+    H, W = wl.H, wl.W
+    for b in range(len(crops)):
+        for k in range(wl.K):
+            if valid[b, k]:
+                p = int(idx[b, k])
+                assert xy[b, k, 0] == np.float32(2 * (p % W) + 1 - W) / np.float32(W)
+                assert xy[b, k, 1] == np.float32(2 * (p // W) + 1 - H) / np.float32(H)
+
+
+def test_workload4_planted_peaks_recovered():
+    wl, head = run_config(4)
+    idx = head.idx.cpu().numpy()
+    centres = wl.extra["centres"]
+    hits = 0
+    total = 0
+    for b in range(0, wl.B, 7):
+        for k in range(17):
+            p = int(idx[b, k])
+            u, v = centres[b, k]
+            total += 1
+            hits += abs(p % 96 - (4 * u - 0.5)) <= 2.5 and abs(p // 96 - (4 * v - 0.5)) <= 2.5
+    # noise N(0, 0.5^2) and neighbouring bumps can move a few peaks; the bulk must sit on the plant
+    assert hits / total > 0.9, hits / total
+
+
+# ----------------------------------------------------------------------------- failure path
+def test_bounded_wait_timeout_reports_and_recovers():
+    wl = S.make_case(51, 2, 24, 24, 128, 17, 2, kern_dtype="bf16", valid="all")
+    kern = S.random_bf16_rows(51, (wl.Bk, wl.M, wl.K, wl.C), 1.0 / np.sqrt(wl.C))
+    gk.gkd_set_wait_timeout_ms(200)
+    try:
+        gk.gkd_debug_set_flags(gk.DEBUG_SKIP_PRODUCER_ARRIVE)
+        feat = to_dev(wl.feat)
+        kd = bf16_dev(kern)
+        heat = torch.empty((wl.B, wl.M, wl.K, 96, 96), device=dev())
+        gk.gkd_heatmap(feat, gk.GKD_F32, wl.B, 24, 24, wl.C, 4, kd, gk.GKD_BF16, wl.M * wl.K * wl.C,
+                       to_dev(wl.mask), wl.M * wl.K, wl.M, wl.K, heat)
+        with pytest.raises(gk.GkdError) as e:
+            gk.gkd_check_device_error()
+        assert e.value.status == gk.GKD_ERR_TIMEOUT
+    finally:
+        gk.gkd_debug_set_flags(0)
+        gk.gkd_set_wait_timeout_ms(2000)
+    # the context is still usable and the next launch is correct
+    got = run_heatmap(wl, kern)
+    ref = O.heatmaps(feat64(wl), O.bf16_decode(kern), wl.mask, 4, "bf16")
+    g, _ = valid_heat_rows(got, wl.mask)
+    r, _ = valid_heat_rows(ref, wl.mask)
+    assert_rows_close(g, r, BF16_TOL, "after timeout")
+
+
+def test_rejects_host_pointer():
+    host = torch.zeros(1024)
+    with pytest.raises(gk.GkdError) as e:
+        gk.gkd_norm_kernels(host, to_dev(np.ones(8, np.uint8)), 1, 1, 8, 128, 1e-12, gk.GKD_F32,
+                            torch.empty(1024, device=dev()))
+    assert e.value.status in (gk.GKD_ERR_ARG, gk.GKD_ERR_CUDA)
