@@ -1,0 +1,377 @@
+"""Benchmark of the GKDT detection head on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gkd|reference] [--config 2]
+
+One step = the whole head over one batch of the workload: gkd_norm_kernels ->
+gkd_heatmap (fused 4x upsample + 1x1 contraction on tcgen05) ->
+gkd_fuse_decode (plus gkd_pool_prototypes on workloads whose visual rows are
+pooled). The default workload (2) is a GKDT-L-shaped batch of 64 crops,
+C = 1024, 24x24 -> 96x96, dual prompts padded to 80 rows with U{5..80} valid.
+
+For N > 1 (launched by torch.distributed.run) every rank runs its own batch
+(weak scaling: crops are independent, no collective on the data path); the
+time is the max over ranks. Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the plain fp64 restatement of the head)
+on the host cores, on the same workload, each step a bounded sample of it.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "heatmap-head crops/sec (C=1024, 80 prompts, 96×96) and % of roofline, 1 B200"
+UNIT = "crops/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["gkd", "reference"], default="gkd")
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "MEASURED_PEAKS.json"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for name in ("heatmap_tc.cu", "ptx.cuh", "gkd_internal.h"):
+        with open(os.path.join(ROOT, "prompt_conditioned_keypoint_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(cfg: int):
+    """DRAM bytes per heatmap launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = t.get(f"workload{cfg}")
+    if not ent or ent.get("kernel_source_digest") != kernel_source_digest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls NVML (the source nvidia-smi reads) during the timed region."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period = index, period_s
+        self.samples = []
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:   # no NVML: report it, do not guess
+            self.err = str(e)
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return fn(self.h)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((sm, self._reasons(), util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": f"nvml unavailable: {self.err}"}
+        busy = [s for s in self.samples if not (s[1] & 0x1)] or self.samples
+        bits = 0
+        for s in busy:
+            bits |= s[1]
+        return {"sm_mhz": statistics.median([s[0] for s in busy]) if busy else None, "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if bits & b and b != 0x1],
+                "samples": len(busy)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+def oracle_sample(wl, crop: int, out_rows=None):
+    """The oracle head on one crop (optionally a band of output rows)."""
+    from oracle import gkd_oracle as O
+    f = O.bf16_decode(wl.feat[crop:crop + 1]) if wl.feat_dtype == "bf16" else wl.feat[crop:crop + 1].astype(np.float64)
+    kb = 0 if wl.Bk == 1 else crop
+    if wl.support is not None:
+        proto = O.pool_prototypes(wl.support[crop:crop + 1], wl.kpts[crop:crop + 1], wl.kmask[crop:crop + 1],
+                                  wl.sigma, wl.stride)
+        rows = np.zeros((1, wl.M, wl.K, wl.C))
+        rows[:, 0] = proto
+        if wl.M == 2:
+            rows[:, 1] = wl.rows[crop:crop + 1, 1]
+    else:
+        rows = wl.rows[kb:kb + 1].astype(np.float64)
+    mask = wl.mask[kb:kb + 1]
+    khat = O.norm_rows(rows, mask)
+    if wl.kern_dtype == "bf16":
+        khat = O.bf16_round(khat)
+    heat = O.heatmap_crop(f[0], khat[0], mask[0], wl.up, wl.kern_dtype, out_rows=out_rows)
+    return O.fuse_decode(np.nan_to_num(heat, nan=0.0)[None], mask)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, budget_s: float):
+    """The oracle as it stands on full crops until the time budget is spent."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_sample(wl, n % wl.B)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= wl.B:
+            break
+    return {"value": n / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} full crop(s) of the same workload, fp64 numpy oracle, {el:.1f} s wall"}
+
+
+def run_reference(args, cfg_desc):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    from prompt_conditioned_keypoint_b200 import synthetic as S
+    wl = S.make_config(args.config)
+    H = wl.H
+    # size the per-step sample (a band of output rows of one crop) so the whole run stays near two minutes
+    t0 = time.perf_counter()
+    oracle_sample(wl, 0)
+    t_crop = time.perf_counter() - t0
+    total_steps = args.steps + args.warmup
+    frac = min(1.0, 120.0 / max(total_steps * t_crop, 1e-9))
+    nrows = max(1, min(H, int(math.floor(frac * H))))
+    sel = list(range(nrows))
+    for i in range(args.warmup):
+        oracle_sample(wl, i % wl.B, sel)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_sample(wl, i % wl.B, sel)
+    el = time.perf_counter() - t0
+    crops = args.steps * nrows / H
+    value = crops / el
+    sample = f"per step: output rows 0..{nrows - 1} of one crop ({nrows}/{H} of its pixels), fp64 numpy oracle"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": cfg_desc,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def main(argv=None):
+    args = parse_args(argv)
+    rank, local_rank, world = dist_env()
+    from prompt_conditioned_keypoint_b200 import synthetic as S
+    cfg_desc = {"workload": S.CONFIG_NAMES[args.config], "workload_id": args.config}
+    if args.impl == "reference":
+        return run_reference(args, cfg_desc)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    import torch
+    from prompt_conditioned_keypoint_b200 import binding as gk
+    from prompt_conditioned_keypoint_b200.head import GkdHead, HeadShape
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    wl = S.make_config(args.config, shard=rank)
+    shape = HeadShape.of(wl)
+    head = GkdHead(shape, dev)
+    host = head.host_inputs(wl, pin=True)
+    stream = torch.cuda.Stream(dev)
+    head.upload(host, stream)
+    stream.synchronize()
+
+    def barrier():
+        if pg:
+            pg.barrier()
+
+    # warm-up
+    for _ in range(args.warmup):
+        head.forward(stream)
+    stream.synchronize()
+    gk.gkd_check_device_error(stream)
+
+    # timed region: exactly K steps, events on the launching stream
+    ev_hm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        head.forward(stream, heatmap_events=ev_hm[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier()
+    gk.gkd_check_device_error(stream)
+    elapsed_s = t_start.elapsed_time(t_end) / 1e3
+    hm_s = sum(a.elapsed_time(b) for a, b in ev_hm) / 1e3 / args.steps
+
+    t = torch.tensor([elapsed_s], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    max_s = float(t.item())
+    value = world * shape.B * args.steps / max_s
+
+    # roofline of the dominant kernel (gkd_heatmap)
+    peaks, peak_src = measured_peaks()
+    flops = head.algorithmic_heatmap_flops(wl.mask)
+    achieved = flops / hm_s / 1e12
+    elt = 2 if shape.feat_dtype == "bf16" else 4
+    rows_valid = float(wl.mask.reshape(wl.mask.shape[0], -1).sum(1).sum()) * (shape.B if shape.shared else 1)
+    hbm_bytes = shape.B * shape.h * shape.w * shape.C * elt + rows_valid * shape.C * 2 / (shape.B if shape.shared else 1) \
+        + rows_valid * shape.H * shape.W * 4
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = hbm_bytes / (peaks["hbm_gbs"] * 1e9)
+    if shape.kern_dtype == "bf16":
+        bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    else:
+        bound = "alu"
+    if bound == "tensor":
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"]}
+    elif bound == "hbm":
+        ach = hbm_bytes / hm_s / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"]}
+    else:
+        peak_alu = 148 * 128 * 2 * 1.965e3 / 1e3   # fp32 FMA lanes x 2 flop x max clock, TFLOP/s
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s", "frac": achieved / peak_alu}
+    traffic = committed_traffic(args.config)
+    roof.update({"traffic": traffic, "kernel": "gkd_heatmap", "peak_source": f"{peak_src} (burst figure)",
+                 "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": hbm_bytes,
+                 "launch_us": hm_s * 1e6, "roofline_us": max(t_tensor, t_hbm) * 1e6,
+                 "frac_of_kernel_roofline": max(t_tensor, t_hbm) / hm_s if bound != "alu" else None})
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": shape.kern_dtype, "data": "synthetic",
+            "config": dict(cfg_desc, crops_per_gpu=shape.B, global_batch=world * shape.B, C=shape.C, K=shape.K,
+                           M=shape.M, grid=f"{shape.h}x{shape.w}->{shape.H}x{shape.W}",
+                           parallelism=f"dp{world} (crops sharded, no data-path collective)",
+                           l2="inputs larger than L2 (features + heatmaps per step exceed 126 MB)"),
+            "heatmap_gflops": flops / hm_s / 1e9, "roofline": roof,
+            "gpu_launches": args.steps * shape.launches_per_step(), "clocks": clocks.summary()}
+
+    # end to end through the public API: pinned host inputs in, decoded keypoints out
+    if not args.no_e2e:
+        outh = None
+        for _ in range(3):
+            outh = head.run_host(host, outh, stream)
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            outh = head.run_host(host, outh, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
+        if pg:
+            pg.all_reduce(te, op=pg.ReduceOp.MAX)
+        line["e2e"] = {"value": world * shape.B * args.e2e_steps / float(te.item()), "unit": UNIT,
+                       "h2d_bytes_per_step": head.host_input_bytes(host), "d2h_bytes_per_step": head.output_bytes(),
+                       "steps": args.e2e_steps}
+    gk.gkd_check_device_error(stream)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

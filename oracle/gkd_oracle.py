@@ -143,11 +143,14 @@ def interp_matrix(n: int, up: int) -> np.ndarray:
     return R
 
 
-def upsample(feat: np.ndarray, up: int = 4) -> np.ndarray:
-    """U[Y,X,c] = sum_i sum_j Ry[Y,i] Rx[X,j] F[i,j,c]; feat [h][w][C] -> [H][W][C] float64."""
+def upsample(feat: np.ndarray, up: int = 4, out_rows=None) -> np.ndarray:
+    """U[Y,X,c] = sum_i sum_j Ry[Y,i] Rx[X,j] F[i,j,c]; feat [h][w][C] -> [H][W][C] float64.
+    `out_rows` restricts the result to those output rows Y (in that order)."""
     F = np.asarray(feat, dtype=np.float64)
     h, w, C = F.shape
     Ry = interp_matrix(h, up)
+    if out_rows is not None:
+        Ry = Ry[list(out_rows)]
     Rx = interp_matrix(w, up)
     tmp = np.einsum("Xj,ijc->iXc", Rx, F)       # along x
     return np.einsum("Yi,iXc->YXc", Ry, tmp)    # then along y
@@ -157,13 +160,14 @@ def upsample(feat: np.ndarray, up: int = 4) -> np.ndarray:
 # a4: 1x1 dynamic-kernel contraction
 # ----------------------------------------------------------------------------
 def heatmap_crop(feat: np.ndarray, kern: np.ndarray, mask: np.ndarray, up: int = 4,
-                 operand: str = "f32") -> np.ndarray:
+                 operand: str = "f32", out_rows=None) -> np.ndarray:
     """heat[m,k,Y,X] = sum_c kern[m,k,c] * U[Y,X,c] for valid rows (NaN elsewhere).
 
     feat [h][w][C] and kern [M][K][C] hold the stored operand values (already
     widened to float64). operand == "bf16": U is rounded to bf16 before the
-    contraction (the kernel rows are bf16 already); the sum is float64."""
-    U = upsample(feat, up)
+    contraction (the kernel rows are bf16 already); the sum is float64.
+    `out_rows` restricts the heatmaps to those output rows."""
+    U = upsample(feat, up, out_rows)
     if operand == "bf16":
         U = bf16_round(U)
     H, W, C = U.shape

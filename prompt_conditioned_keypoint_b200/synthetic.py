@@ -69,8 +69,12 @@ class Workload:
         return self.up * self.w
 
 
+_SHARD = 0   # data shard of the calling process (set by make_config's `shard`)
+
+
 def _rng(cfg_seed: int, purpose: int, b: int = 0) -> np.random.Generator:
-    ss = np.random.SeedSequence(entropy=cfg_seed, spawn_key=(purpose, b))
+    key = (purpose, b) if _SHARD == 0 else (purpose, b, _SHARD)
+    ss = np.random.SeedSequence(entropy=cfg_seed, spawn_key=key)
     return np.random.Generator(np.random.PCG64(ss))
 
 
@@ -113,9 +117,20 @@ def _crop_list(B: int, crops) -> list[int]:
     return [int(b) for b in crops]
 
 
-def make_config(cfg: int, crops=None) -> Workload:
+def make_config(cfg: int, crops=None, shard: int = 0) -> Workload:
     """Inputs of workload `cfg` (1..5). `crops` selects a subset of crop indices
-    (the selected crops get exactly the values they have in the full batch)."""
+    (the selected crops get exactly the values they have in the full batch).
+    `shard` > 0 draws an independent batch of the same distribution (one per
+    data-parallel rank); shard 0 is the canonical batch."""
+    global _SHARD
+    _SHARD = int(shard)
+    try:
+        return _make_config(cfg, crops)
+    finally:
+        _SHARD = 0
+
+
+def _make_config(cfg: int, crops) -> Workload:
     seed = 1000 + cfg
     if cfg == 1:
         return _pooled_workload(seed, "cfg1", B=1, h=24, w=24, C=1024, K=80, n_kpts=17,

@@ -402,3 +402,12 @@ def test_head_chain_consistency_small():
                 if mask[b, m, k]:
                     np.testing.assert_allclose(heat[b, m, k], U @ kh[b, m, k], rtol=1e-12)
     assert np.array_equal(valid, (mask.sum(1) > 0).astype(np.uint8))
+
+
+def test_out_rows_selection_is_a_restriction():
+    F = RNG.standard_normal((5, 6, 3))
+    kern = RNG.standard_normal((2, 2, 3))
+    mask = np.ones((2, 2), np.uint8)
+    full = O.heatmap_crop(F, kern, mask, 4, "bf16")
+    part = O.heatmap_crop(F, kern, mask, 4, "bf16", out_rows=[3, 0, 17])
+    np.testing.assert_array_equal(part, full[:, :, [3, 0, 17]])
