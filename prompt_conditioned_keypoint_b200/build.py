@@ -42,12 +42,17 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not verbose_ptxas and not _stale():
+def build(force: bool = False, verbose_ptxas: bool = False, trace_to: str | None = None) -> str:
+    """Build libgkd.so. `trace_to` builds a separate timeline-tracing variant
+    (-DGKD_TRACE, exports gkd_trace_read) at that path instead."""
+    out = trace_to or LIB
+    if trace_to is None and not force and not verbose_ptxas and not _stale():
         return LIB
     cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include"),
-           "-o", LIB + ".tmp", *sources()]
+           "-o", out + ".tmp", *sources()]
+    if trace_to is not None:
+        cmd.insert(1, "-DGKD_TRACE")
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     proc = subprocess.run(cmd, capture_output=True, text=True)
@@ -55,16 +60,17 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + proc.stdout + proc.stderr)
     if verbose_ptxas:
         sys.stderr.write(proc.stdout + proc.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--trace-to", default=None, help="build the tracing variant at this path")
     args = ap.parse_args(argv)
-    print(build(force=args.force, verbose_ptxas=args.verbose_ptxas))
+    print(build(force=args.force, verbose_ptxas=args.verbose_ptxas, trace_to=args.trace_to))
 
 
 if __name__ == "__main__":

@@ -34,15 +34,17 @@ cudaError_t launch_heatmap_f32(const float* feat, int B, int h, int w, int C, co
                                long long kern_batch_stride, const uint8_t* mask, long long mask_batch_stride,
                                int M, int K, float* heat, cudaStream_t stream);
 
+constexpr int kKernMaps = 16;   // kernel-row boxes of 8, 16, ..., 128 rows
+
 struct HeatmapTcArgs {
-  CUtensorMap tmap_feat;     // feature slabs  {C, w, h, B}
-  CUtensorMap tmap_kern8;    // kernel rows, 8-row boxes  {C, K, M, Bk}
-  CUtensorMap tmap_kern32;   // kernel rows, 32-row boxes
+  CUtensorMap tmap_feat;                 // feature slabs: fp32 {32, w, h, C/32, B} or {C, w, h, B}
+  CUtensorMap tmap_kern[kKernMaps];      // kernel rows {C, K, M, Bk}, box {64, 8 (i + 1), 1, 1}
   const uint8_t* mask;
   long long mask_batch_stride;
   float* heat;
   int B, h, w, C, M, K;
   int feat_bf16;
+  int feat_5d;               // fp32 slab as one 5-D box (C % 32 == 0), else two 4-D boxes
   int kern_shared;           // kernels shared by all crops (batch stride 0)
   unsigned* err;             // device error word
   unsigned long long wait_limit_ns;

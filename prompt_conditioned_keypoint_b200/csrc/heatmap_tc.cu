@@ -9,50 +9,64 @@
 // N = the crop's valid prompt rows, K = channels. Operands are bf16, the sum is
 // fp32 in tensor memory.
 //
-// Persistent kernel, one CTA per SM, 14 warps:
-//   warp 0      TMA: per 64-channel chunk, a 3x10-patch feature slab (128B
-//               swizzled) and the crop's kernel-row segments (the B operand);
-//   warp 1      MMA issuer: tcgen05.mma kind::f16, A from TMEM, B from smem;
-//   warps 2-5   epilogue: tcgen05.ld of the accumulators, heatmap stores;
-//   warps 6-13  upsample producers: each thread owns a vertical pixel pair
-//               sharing the same four source taps, lerps in fp32 (packed f32x2),
-//               rounds to bf16 and writes the A operand straight into TMEM with
-//               tcgen05.st (never through shared memory).
-// A work unit is 8 output rows x 32 output columns (256 pixels = two M=128
-// tiles that share the B operand). Units are split over CTAs by a static
-// cost-balanced partition computed in the prologue. Every wait is bounded; a
-// timeout sets the device error word and all roles drain and exit.
-#include <cstdio>
-
+// Persistent kernel, one CTA per SM, 14 warps, one M=128 tile (4 output rows x
+// 32 output columns, which all read the same two source rows) per work unit:
+//   warp 0       TMA: per 64-channel chunk, a 2x10-patch feature slab (128B
+//                swizzled) and one box of kernel rows per modality (the B
+//                operand) into a 6-stage ring;
+//   warp 1       MMA issuer: tcgen05.mma kind::f16, A from tensor memory, B from
+//                shared memory, into one of two accumulator buffers, so the next
+//                unit accumulates while the epilogue drains the last one;
+//   warps 2-5    epilogue: tcgen05.ld of the accumulator, transpose through a
+//                padded shared tile, coalesced float4 heatmap rows;
+//   warps 6-13   upsample producers: a thread owns one output column of four
+//                pixels (one x-lerp per source row serves all four), lerps in
+//                fp32 (packed f32x2), rounds to bf16 and writes the A operand
+//                straight into tensor memory with tcgen05.st.16x256b.
+// Units are split over CTAs by a static cost-balanced partition computed in the
+// prologue. Every wait is bounded; a timeout sets the device error word and all
+// roles drain their in-flight copies and MMAs and exit.
 #include "gkd_internal.h"
 #include "ptx.cuh"
 
 namespace gkd {
 namespace tc {
 
-constexpr int kStages = 3;
+// Optional timeline tracing (build with -DGKD_TRACE): CTA 0 records %globaltimer
+// at each hand-off between roles; read back with gkd_trace_read().
+#ifdef GKD_TRACE
+__device__ unsigned long long g_trace[16][2048];
+#define GKD_TR(kind, idx) \
+  do { if (blockIdx.x == 0 && (idx) < 2048u) g_trace[kind][idx] = global_timer_ns(); } while (0)
+#else
+#define GKD_TR(kind, idx) do { } while (0)
+#endif
+
+constexpr int kStages = 6;                       // ring: slab + kernel rows (smem), A operand (tmem)
 constexpr int kChunk = 64;                       // channels per K-chunk
 constexpr int kMaxN = 160;                       // accumulator columns per tile
-constexpr int kUnitRows = 8, kUnitCols = 32;
-constexpr int kSlabRows = 3, kSlabCols = 10;
-constexpr int kSlabHalf = 4096;                  // 30 lines x 128 B, padded to 1 KB multiple
-constexpr int kSlabBytes = 2 * kSlabHalf;
+constexpr int kUnitRows = 4, kUnitCols = 32;     // one M=128 tile: 4 output rows x 32 output columns
+constexpr int kSlabRows = 2, kSlabCols = 10, kSlabLines = kSlabRows * kSlabCols;
+constexpr int kSlabBytes = 8192;                 // fp32: two halves (at 0 and 2560, or 0 and 4096); bf16: one
 constexpr int kBBytes = kMaxN * 128;
 constexpr int kStageBytes = kSlabBytes + kBBytes;  // 28 KB, 1 KB aligned
+constexpr int kEpiCols = 16;                     // accumulator columns per epilogue group
+constexpr int kEpiStride = 40;                   // floats per (column, row) line of the epilogue tile
+constexpr int kEpiBufBytes = kEpiCols * kUnitRows * kEpiStride * 4;   // 10 KB
 constexpr int kNumWarps = 14, kThreads = kNumWarps * 32;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpProd0 = 6;   // warps 2-5: epilogue
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kWarpProd0 = 6;
 constexpr int kNumProdWarps = 8, kNumEpiWarps = 4;
+constexpr int kEpiBarrier = 1;                   // named barrier of the four epilogue warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColD0 = 0, kColD1 = kMaxN, kColA = 2 * kMaxN;   // A stages at 320, 384, 448
-constexpr int kCostBias = 48;                    // per-unit cost model: N + bias
-constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + 256 + 32 * 1024;  // padded: one CTA per SM
+constexpr uint32_t kColA = 2 * kMaxN;            // accumulators at 0 and 160; A stages at 320 + 32 s
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 2 * kEpiBufBytes + 512;
 
-struct Smem {            // control block placed after the stage buffers
+struct Smem {            // control block placed after the stage and epilogue buffers
   uint64_t full[kStages];
-  uint64_t afull[kStages];
   uint64_t empty[kStages];
-  uint64_t accfull;
-  uint64_t accempty;
+  uint64_t afull[kStages];
+  uint64_t accfull[2];
+  uint64_t accempty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -62,7 +76,7 @@ struct Smem {            // control block placed after the stage buffers
 
 struct CropInfo {
   int n;                 // accumulator columns (multiple of 16), 0 = nothing to do
-  int kmin[2], len[2], off[2];
+  int kmin0, kmin1, len0, len1, off1;
   uint32_t vbits[5];     // bit c of word c/32: column c maps to a valid (m, k) row
 };
 
@@ -71,15 +85,14 @@ __device__ __forceinline__ const uint8_t* crop_mask(const HeatmapTcArgs& a, int 
 }
 
 // Warp-cooperative: valid-row segments of one crop (all lanes get the result).
+// Segment m covers rows [kmin_m, kmin_m + len_m) of modality m (len a multiple of
+// 8) and lands at accumulator columns [off_m, off_m + len_m), off_0 = 0.
 __device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int lane) {
   CropInfo ci;
   const uint8_t* mb = crop_mask(a, b);
-  int off = 0;
+  int kmin[2] = {0, 0}, len[2] = {0, 0};
 #pragma unroll
   for (int m = 0; m < 2; ++m) {
-    ci.kmin[m] = 0;
-    ci.len[m] = 0;
-    ci.off[m] = off;
     if (m >= a.M) continue;
     int first = a.K, last = -1;
     for (int kb = 0; kb < a.K; kb += 32) {
@@ -92,20 +105,25 @@ __device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int
       }
     }
     if (last >= 0) {
-      ci.kmin[m] = first;
-      ci.len[m] = (last - first + 1 + 7) & ~7;
-      off += ci.len[m];
+      kmin[m] = first;
+      len[m] = (last - first + 1 + 7) & ~7;
     }
   }
-  ci.n = (off + 15) & ~15;
+  ci.kmin0 = kmin[0];
+  ci.kmin1 = kmin[1];
+  ci.len0 = len[0];
+  ci.len1 = len[1];
+  ci.off1 = len[0];
+  const int used = len[0] + len[1];
+  ci.n = (used + 15) & ~15;
 #pragma unroll
   for (int g = 0; g < 5; ++g) {
     const int col = g * 32 + lane;
     bool v = false;
-    if (col < off) {
-      const int m = (a.M == 2 && col >= ci.off[1]) ? 1 : 0;
-      const int k = ci.kmin[m] + (col - ci.off[m]);
-      v = (col - ci.off[m] < ci.len[m]) && k < a.K && mb[m * a.K + k] != 0;
+    if (col < used) {
+      const bool m1 = col >= ci.off1;
+      const int k = (m1 ? ci.kmin1 : ci.kmin0) + (col - (m1 ? ci.off1 : 0));
+      v = k < a.K && mb[(m1 ? a.K : 0) + k] != 0;
     }
     ci.vbits[g] = __ballot_sync(0xffffffffu, v);
   }
@@ -127,6 +145,11 @@ __device__ __forceinline__ int crop_n_serial(const HeatmapTcArgs& a, int b) {
   }
   return (off + 15) & ~15;
 }
+
+// Relative cost of one unit with n accumulator columns: the slowest of the
+// upsample producers (independent of n), the kernel-row copy (grows with n)
+// and the MMAs.
+__device__ __forceinline__ long long unit_cost(int n) { return n == 0 ? 0 : max(2 * n + 80, 230); }
 
 __device__ __forceinline__ void src_taps(int d, int n, int& i0, int& i1, float& lam) {
   const float s = fmaxf((static_cast<float>(d) + 0.5f) * 0.25f - 0.5f, 0.0f);
@@ -156,61 +179,86 @@ __device__ __forceinline__ float2 f2sub(float2 b, float2 a) {   // b - a, one ro
   return __ffma2_rn(a, make_float2(-1.f, -1.f), b);
 }
 
-struct PixelPair {
-  int Ya, X;        // upper pixel; the lower one is (Ya + 1, X)
-  int L00, L01, L10, L11;   // slab lines of the four taps
-  float2 lx, la, lb;        // lerp weights (broadcast to both lanes of a float2)
+// Pixel layout of a unit (rows Y0..Y0+3, Y0 = 4 vb - 2; columns X0..X0+31):
+// TMEM lane 32 q + 16 hf + 8 e + j  <->  pixel (Y0 + 2 hf + e, X0 + 8 q + j).
+// All four rows read the same two source rows, so a producer thread owns the
+// whole column of four pixels at one X (lanes j, j+8 of both 16-lane halves).
+struct Column4 {
+  int X;
+  int L[4];                   // slab lines of taps (r0,c0) (r0,c1) (r1,c0) (r1,c1), within a half
+  float2 lx;                  // x weight
+  float2 ly[4];               // y weight of rows Y0 .. Y0+3
 };
 
-__device__ __forceinline__ PixelPair pair_geometry(const HeatmapTcArgs& a, int vb, int ub, int q, int lane) {
-  PixelPair pp;
-  const int Y0 = kUnitRows * vb - 2, X0 = kUnitCols * ub;
-  const int Yg = Y0 + ((q >> 1) << 2);
-  pp.Ya = Yg + 2 * (lane >> 4);
-  pp.X = X0 + ((q & 1) << 4) + (lane & 15);
-  int r0, r1, r0b, r1b, c0, c1;
-  float lya, lyb, lxx;
-  src_taps(pp.Ya, a.h, r0, r1, lya);
-  src_taps(pp.Ya + 1, a.h, r0b, r1b, lyb);
-  src_taps(pp.X, a.w, c0, c1, lxx);
-  // both pixels of the pair read the same two source rows (r0, r1)
-  const int sr0 = r0 - (2 * vb - 1), sr1 = r1 - (2 * vb - 1);
+__device__ __forceinline__ Column4 column_geometry(const HeatmapTcArgs& a, int vb, int ub, int q, int j) {
+  Column4 cg;
+  const int Y0 = kUnitRows * vb - 2;
+  cg.X = kUnitCols * ub + 8 * q + j;
+  int r0 = 0, r1 = 0, c0, c1;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    int i0, i1;
+    float l;
+    src_taps(Y0 + r, a.h, i0, i1, l);
+    r0 = i0;          // the same for all four rows (clamped to 0 on the first band)
+    r1 = i1;
+    cg.ly[r] = make_float2(l, l);
+  }
+  float lxx;
+  src_taps(cg.X, a.w, c0, c1, lxx);
+  // slab rows hold source rows vb-1, vb; on the first band r0 = 0 -> slab row 1 and
+  // every y weight is 0, so the second tap row only needs to stay inside the slab
+  const int sr0 = r0 - (vb - 1);
+  const int sr1 = min(r1 - (vb - 1), 1);
   const int sc0 = c0 - (8 * ub - 1), sc1 = c1 - (8 * ub - 1);
-  pp.L00 = sr0 * kSlabCols + sc0;
-  pp.L01 = sr0 * kSlabCols + sc1;
-  pp.L10 = sr1 * kSlabCols + sc0;
-  pp.L11 = sr1 * kSlabCols + sc1;
-  pp.lx = make_float2(lxx, lxx);
-  pp.la = make_float2(lya, lya);
-  pp.lb = make_float2(lyb, lyb);
-  return pp;
+  cg.L[0] = sr0 * kSlabCols + sc0;
+  cg.L[1] = sr0 * kSlabCols + sc1;
+  cg.L[2] = sr1 * kSlabCols + sc0;
+  cg.L[3] = sr1 * kSlabCols + sc1;
+  cg.lx = make_float2(lxx, lxx);
+  return cg;
 }
 
-__device__ __forceinline__ const uint8_t* swz(const uint8_t* base, int line, int chunk16) {
-  return base + line * 128 + (((chunk16 ^ (line & 7))) << 4);
-}
-
-// Upsample two fp32 channel pairs of a pixel pair; writes packed bf16x2 words.
-__device__ __forceinline__ void lerp_pair(float2 f00, float2 f01, float2 f10, float2 f11, const PixelPair& pp,
-                                          uint32_t& oa, uint32_t& ob) {
-  const float2 t0 = __ffma2_rn(pp.lx, f2sub(f01, f00), f00);
-  const float2 t1 = __ffma2_rn(pp.lx, f2sub(f11, f10), f10);
+// One channel pair of the four-pixel column: x-lerps on both source rows, then
+// four y-lerps; returns the packed bf16x2 words of rows 0..3.
+__device__ __forceinline__ void lerp_column(float2 f00, float2 f01, float2 f10, float2 f11, const Column4& cg,
+                                            uint32_t (&o)[4]) {
+  const float2 t0 = __ffma2_rn(cg.lx, f2sub(f01, f00), f00);
+  const float2 t1 = __ffma2_rn(cg.lx, f2sub(f11, f10), f10);
   const float2 dt = f2sub(t1, t0);
-  const float2 ua = __ffma2_rn(pp.la, dt, t0);
-  const float2 ubv = __ffma2_rn(pp.lb, dt, t0);
-  oa = pack_bf16x2(ua.x, ua.y);
-  ob = pack_bf16x2(ubv.x, ubv.y);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float2 u = __ffma2_rn(cg.ly[r], dt, t0);
+    o[r] = pack_bf16x2(u.x, u.y);
+  }
 }
 
 __device__ __forceinline__ float2 bf16lo_hi(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint2 ld_shared_u2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_constant__ HeatmapTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Smem* ctl = reinterpret_cast<Smem*>(smem + kStages * kStageBytes);
+  uint8_t* epi_buf = smem + kStages * kStageBytes;
+  Smem* ctl = reinterpret_cast<Smem*>(epi_buf + 2 * kEpiBufBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
 
@@ -225,11 +273,13 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ctl->full[s], 1);
-      mbar_init(&ctl->afull[s], kNumProdWarps);
       mbar_init(&ctl->empty[s], 1);
+      mbar_init(&ctl->afull[s], kNumProdWarps);
     }
-    mbar_init(&ctl->accfull, 1);
-    mbar_init(&ctl->accempty, kNumEpiWarps);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctl->accfull[t], 1);
+      mbar_init(&ctl->accempty[t], kNumEpiWarps);
+    }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
     ctl->unit_begin = ~0ull;
@@ -241,10 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     tmem_alloc(&ctl->tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kWarpTma && lane == 0) {
-    tma_prefetch_desc(&a.tmap_feat);
-    tma_prefetch_desc(&a.tmap_kern8);
-    tma_prefetch_desc(&a.tmap_kern32);
+  if (warp == kWarpTma && lane < 1 + kKernMaps) {
+    tma_prefetch_desc(lane == 0 ? &a.tmap_feat : &a.tmap_kern[lane - 1]);
   }
   __syncthreads();
 
@@ -253,8 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   if (a.kern_shared && a.mask_batch_stride == 0) {
     // every crop has the same rows: split the units evenly
     if (tid == 0) {
-      const int n0 = crop_n_serial(a, 0);
-      if (n0 == 0) {
+      if (crop_n_serial(a, 0) == 0) {
         ctl->unit_begin = ctl->unit_end = 0;
       } else {
         ctl->unit_begin = (total_units * g + G - 1) / G;
@@ -264,10 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   } else {
     // pass 1: total cost
     long long local = 0;
-    for (int b = tid; b < a.B; b += kThreads) {
-      const int n = crop_n_serial(a, b);
-      if (n) local += (n + kCostBias) * nU;
-    }
+    for (int b = tid; b < a.B; b += kThreads) local += unit_cost(crop_n_serial(a, b)) * nU;
     for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
     if (lane == 0 && local) atomicAdd(reinterpret_cast<unsigned long long*>(&ctl->total_cost),
                                       static_cast<unsigned long long>(local));
@@ -279,8 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     long long carry = 0;
     for (int base = 0; base < a.B; base += kThreads) {
       const int b = base + tid;
-      const int n = (b < a.B) ? crop_n_serial(a, b) : 0;
-      const long long c = n ? (n + kCostBias) : 0;
+      const long long c = (b < a.B) ? unit_cost(crop_n_serial(a, b)) : 0;
       const long long tot = c * nU;
       long long incl = tot;
       for (int o = 1; o < 32; o <<= 1) {
@@ -318,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   const unsigned long long ubeg = ctl->unit_begin, uend = ctl->unit_end;
   const uint64_t lim = a.wait_limit_ns;
   volatile int* abortp = &ctl->abort_flag;
+  const uint32_t smem_base = smem_u32(smem);
 
   if (warp == kWarpTma) {
     // ---------------------------------------------------------------- TMA
@@ -325,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
+    const uint32_t slab_bytes = (a.feat_bf16 ? 1 : 2) * kSlabLines * 128;
     for (unsigned long long u = ubeg; u < uend && ok; ++u) {
       const int b = static_cast<int>(u / nU), j = static_cast<int>(u % nU);
       if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
@@ -340,38 +385,35 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
           break;
         }
         if (lane == 0) {
+          GKD_TR(0, it);
           uint8_t* st = smem + s * kStageBytes;
-          const uint32_t bytes = (a.feat_bf16 ? kSlabRows * kSlabCols * 128 : 2 * kSlabRows * kSlabCols * 128) +
-                                 (ci.len[0] + ci.len[1]) * 128;
-          mbar_arrive_expect_tx(&ctl->full[s], bytes);
+          mbar_arrive_expect_tx(&ctl->full[s], slab_bytes + (ci.len0 + ci.len1) * 128);
           const int c0 = ch * kChunk;
           if (a.feat_bf16) {
-            tma_load_4d(st, &a.tmap_feat, &ctl->full[s], c0, 8 * ub - 1, 2 * vb - 1, b);
+            tma_load_4d(st, &a.tmap_feat, &ctl->full[s], c0, 8 * ub - 1, vb - 1, b);
+          } else if (a.feat_5d) {
+            tma_load_5d(st, &a.tmap_feat, &ctl->full[s], 0, 8 * ub - 1, vb - 1, c0 / 32, b);
           } else {
-            tma_load_4d(st, &a.tmap_feat, &ctl->full[s], c0, 8 * ub - 1, 2 * vb - 1, b);
-            tma_load_4d(st + kSlabHalf, &a.tmap_feat, &ctl->full[s], c0 + 32, 8 * ub - 1, 2 * vb - 1, b);
+            tma_load_4d(st, &a.tmap_feat, &ctl->full[s], c0, 8 * ub - 1, vb - 1, b);
+            tma_load_4d(st + 4096, &a.tmap_feat, &ctl->full[s], c0 + 32, 8 * ub - 1, vb - 1, b);
           }
           uint8_t* bdst = st + kSlabBytes;
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const int len = ci.len[m], off = ci.off[m], kmin = ci.kmin[m];
-            int r = 0;
-            for (; len - r >= 32; r += 32)
-              tma_load_4d(bdst + (off + r) * 128, &a.tmap_kern32, &ctl->full[s], c0, kmin + r, m, bk);
-            for (; r < len; r += 8)
-              tma_load_4d(bdst + (off + r) * 128, &a.tmap_kern8, &ctl->full[s], c0, kmin + r, m, bk);
-          }
+          if (ci.len0) tma_load_4d(bdst, &a.tmap_kern[(ci.len0 >> 3) - 1], &ctl->full[s], c0, ci.kmin0, 0, bk);
+          if (ci.len1)
+            tma_load_4d(bdst + ci.off1 * 128, &a.tmap_kern[(ci.len1 >> 3) - 1], &ctl->full[s], c0, ci.kmin1, 1, bk);
+          GKD_TR(1, it);
         }
         __syncwarp();
       }
     }
-    // drain: make sure no load issued by this warp is still landing in shared memory
+    // drain: no load issued by this warp may still be landing in shared memory
     if (lane == 0) {
       for (uint32_t k = 0; k < kStages && k < it; ++k) {
         const uint32_t last = it - 1 - k;
         if (!mbar_wait_drain(&ctl->full[last % kStages], (last / kStages) & 1, lim)) atomicOr(a.err, kErrTimeout);
       }
     }
+    __syncwarp();
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA
     uint32_t it = 0, v = 0;
@@ -383,42 +425,52 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
       if (ci.n == 0) continue;
       const uint32_t idesc = make_idesc(ci.n);
-      if (v > 0 && !mbar_wait_bounded(&ctl->accempty, (v - 1) & 1, lim, abortp)) {
+      const int buf = v & 1;
+      const uint32_t dcol = tmem + buf * kMaxN;
+      if (v >= 2 && !mbar_wait_bounded(&ctl->accempty[buf], ((v >> 1) & 1) ^ 1, lim, abortp)) {
         if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
         ok = false;
         break;
       }
+      if (lane == 0) GKD_TR(13, v);
       tc_fence_after();
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
         const int s = it % kStages;
         const uint32_t par = (it / kStages) & 1;
-        if (!mbar_wait_bounded(&ctl->full[s], par, lim, abortp) ||
-            !mbar_wait_bounded(&ctl->afull[s], par, lim, abortp)) {
+        if (lane == 0) GKD_TR(4, it);
+        const bool okf = mbar_wait_bounded(&ctl->full[s], par, lim, abortp);
+        if (lane == 0) GKD_TR(5, it);
+        if (!okf || !mbar_wait_bounded(&ctl->afull[s], par, lim, abortp)) {
           if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
           ok = false;
           break;
         }
+        if (lane == 0) GKD_TR(11, it);
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t bbase = smem_u32(smem + s * kStageBytes + kSlabBytes);
-          const uint32_t acol = kColA + s * 64;
+          GKD_TR(2, it);
+          const uint32_t bbase = smem_base + s * kStageBytes + kSlabBytes;
+          const uint32_t acol = tmem + kColA + s * 32;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = make_bdesc(bbase + kk * 32);
-            const uint32_t acc = (ch > 0 || kk > 0) ? 1u : 0u;
-            umma_ts_f16(tmem + kColD0, tmem + acol + kk * 8, bd, idesc, acc);
-            umma_ts_f16(tmem + kColD1, tmem + acol + 32 + kk * 8, bd, idesc, acc);
+            umma_ts_f16(dcol, acol + kk * 8, make_bdesc(bbase + kk * 32), idesc, (ch > 0 || kk > 0) ? 1u : 0u);
+            if (kk == 0) GKD_TR(12, it);
           }
+          GKD_TR(15, it);
           umma_commit(&ctl->empty[s]);
+          GKD_TR(3, it);
         }
         __syncwarp();
       }
       if (!ok) break;
-      if (lane == 0) umma_commit(&ctl->accfull);
+      if (lane == 0) {
+        umma_commit(&ctl->accfull[buf]);
+        GKD_TR(14, v);
+      }
       __syncwarp();
       ++v;
     }
-    // drain: wait until every MMA issued by this thread has completed
+    // drain: every MMA issued by this thread has completed before teardown
     if (lane == 0 && it > 0) {
       umma_commit(&ctl->drain);
       if (!mbar_wait_drain(&ctl->drain, 0, lim)) atomicOr(a.err, kErrTimeout);
@@ -426,60 +478,83 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     __syncwarp();
   } else if (warp < kWarpProd0) {
     // ---------------------------------------------------------------- epilogue
+    // TMEM -> registers -> padded shared tile [column][row][X] -> float4 rows of the heatmaps
     const int q = warp & 3;
-    uint32_t v = 0;
+    const int et = tid - kWarpEpi0 * 32;           // 0..127
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    const int my_row = 2 * (lane >> 4) + ((lane >> 3) & 1), my_x = 8 * q + (lane & 7);
+    const uint32_t epi_base = smem_u32(epi_buf);
+    uint32_t v = 0, grp = 0;
     int cur_b = -1;
     CropInfo ci{};
-    for (unsigned long long u = ubeg; u < uend; ++u) {
+    bool ok = true;
+    for (unsigned long long u = ubeg; u < uend && ok; ++u) {
       const int b = static_cast<int>(u / nU), j = static_cast<int>(u % nU);
       if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
       if (ci.n == 0) continue;
-      if (!mbar_wait_bounded(&ctl->accfull, v & 1, lim, abortp)) {
+      const int buf = v & 1;
+      if (!mbar_wait_bounded(&ctl->accfull[buf], (v >> 1) & 1, lim, abortp)) {
         if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
+        ok = false;
         break;
       }
       tc_fence_after();
-      const PixelPair pp = pair_geometry(a, j / ncb, j % ncb, q, lane);
-      const bool xin = pp.X < W;
-      const bool ya_in = pp.Ya >= 0 && pp.Ya < H, yb_in = pp.Ya + 1 >= 0 && pp.Ya + 1 < H;
+      if (lane == 0 && warp == kWarpEpi0) GKD_TR(9, v);
+      const int Y0 = kUnitRows * (j / ncb) - 2, X0 = kUnitCols * (j % ncb);
       float* hb = a.heat + static_cast<long long>(b) * a.M * a.K * P;
-      const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
-      for (int n0 = 0; n0 < ci.n; n0 += 16) {
+      const int shift0 = ci.kmin0, shift1 = a.K + ci.kmin1 - ci.off1;
+      const int ngroups = ci.n / kEpiCols;
+      for (int gi = 0; gi < ngroups; ++gi) {
+        const int n0 = gi * kEpiCols;
         uint32_t word = ci.vbits[0];
 #pragma unroll
         for (int g2 = 1; g2 < 5; ++g2)
           if ((n0 >> 5) == g2) word = ci.vbits[g2];
-        const uint32_t bits16 = (word >> (n0 & 31)) & 0xFFFFu;
-        if (bits16 == 0) continue;
-        uint32_t v0[16], v1[16];
-        tmem_ld_32x32b_x16(tmem + lane_off + kColD0 + n0, v0);
-        tmem_ld_32x32b_x16(tmem + lane_off + kColD1 + n0, v1);
+        const uint32_t bits = (word >> (n0 & 31)) & 0xFFFFu;
+        uint32_t vv[16];
+        tmem_ld_32x32b_x16(tmem + lane_off + buf * kMaxN + n0, vv);
         tmem_wait_ld();
+        if (gi == ngroups - 1) {   // accumulator fully read: let the MMA reuse it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->accempty[buf]);
+        }
+        if (bits == 0) continue;   // uniform across the four warps (same crop)
+        // stage this thread's pixel: [col][row][X], row stride kEpiStride floats
+        const uint32_t sb = epi_base + (grp & 1) * kEpiBufBytes;
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int col = n0 + jj;
-          if (!((bits16 >> jj) & 1u)) continue;
-          const bool m1 = a.M == 2 && col >= ci.off[1];
-          const int m = m1 ? 1 : 0;
-          const int k = (m1 ? ci.kmin[1] : ci.kmin[0]) + (col - (m1 ? ci.off[1] : 0));
-          float* row = hb + (static_cast<long long>(m) * a.K + k) * P;
-          if (xin) {
-            if (ya_in) __stcs(row + static_cast<long long>(pp.Ya) * W + pp.X, __uint_as_float(v0[jj]));
-            if (yb_in) __stcs(row + static_cast<long long>(pp.Ya + 1) * W + pp.X, __uint_as_float(v1[jj]));
+        for (int c = 0; c < kEpiCols; ++c)
+          st_shared_f32(sb + ((c * kUnitRows + my_row) * kEpiStride + my_x) * 4, vv[c]);
+        named_bar_sync(kEpiBarrier, kNumEpiWarps * 32);
+        // each thread writes 4 float4 (4 consecutive X of one column and row)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int f = i * 128 + et;
+          const int c = f >> 5, r = (f >> 3) & 3, x4 = f & 7;
+          if ((bits >> c) & 1u) {
+            const int Y = Y0 + r, X = X0 + 4 * x4;
+            if (Y >= 0 && Y < H && X < W) {
+              const float4 val = ld_shared_f4(sb + ((c * kUnitRows + r) * kEpiStride + 4 * x4) * 4);
+              const int n = n0 + c;
+              const int row = n + (n < ci.off1 ? shift0 : shift1);
+              __stcs(reinterpret_cast<float4*>(hb + static_cast<long long>(row) * P + static_cast<long long>(Y) * W + X),
+                     val);
+            }
           }
         }
+        ++grp;   // staging buffers alternate only between groups that passed the barrier
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->accempty);
+      if (lane == 0 && warp == kWarpEpi0) GKD_TR(10, v);
       ++v;
     }
   } else {
     // ---------------------------------------------------------------- upsample producers
     const int q = warp & 3;
     const int hsel = (warp - kWarpProd0) >> 2;   // which 32 channels of each chunk
-    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    const int jx = lane >> 2, cq = lane & 3;      // column within the quadrant, channel quarter
     const bool skip_first = (a.debug_flags & kDbgSkipProducerArrive) != 0;
+    // line offset of this thread's channel half within a stage's slab
+    const int half_lines = a.feat_bf16 ? 0 : (a.feat_5d ? kSlabLines : 32);
     uint32_t it = 0;
     int cur_b = -1;
     CropInfo ci{};
@@ -488,7 +563,15 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       const int b = static_cast<int>(u / nU), j = static_cast<int>(u % nU);
       if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
       if (ci.n == 0) continue;
-      const PixelPair pp = pair_geometry(a, j / ncb, j % ncb, q, lane);
+      const Column4 cg = column_geometry(a, j / ncb, j % ncb, q, jx);
+      // per tap: byte offset of its line inside a stage, and its swizzle pattern
+      uint32_t loff[4], lxs[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int line = hsel * half_lines + cg.L[k];
+        loff[k] = static_cast<uint32_t>(line) * 128u;
+        lxs[k] = static_cast<uint32_t>(line & 7) << 4;
+      }
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
         const int s = it % kStages;
         const uint32_t use = it / kStages;
@@ -499,50 +582,51 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
           break;
         }
         tc_fence_after();
-        const uint8_t* slab = smem + s * kStageBytes;
-        const uint32_t acol = tmem + lane_off + kColA + s * 64 + hsel * 16;
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {      // two halves of 16 channels: 8 TMEM columns each
-          uint32_t oa[8], ob[8];
-          if (!a.feat_bf16) {
-            const uint8_t* half = slab + hsel * kSlabHalf;
+        if (lane == 0 && warp == kWarpProd0) GKD_TR(6, it);
+        const uint32_t st = smem_base + s * kStageBytes;
+        // o[p][r]: channel pair p (4cq, 4cq+2, 16+4cq, 18+4cq of this warp's 32 channels), row r
+        uint32_t o[4][4];
+        if (!a.feat_bf16) {
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const int g4 = hh * 4 + g;
-              const float4 f00 = *reinterpret_cast<const float4*>(swz(half, pp.L00, g4));
-              const float4 f01 = *reinterpret_cast<const float4*>(swz(half, pp.L01, g4));
-              const float4 f10 = *reinterpret_cast<const float4*>(swz(half, pp.L10, g4));
-              const float4 f11 = *reinterpret_cast<const float4*>(swz(half, pp.L11, g4));
-              lerp_pair(make_float2(f00.x, f00.y), make_float2(f01.x, f01.y), make_float2(f10.x, f10.y),
-                        make_float2(f11.x, f11.y), pp, oa[2 * g], ob[2 * g]);
-              lerp_pair(make_float2(f00.z, f00.w), make_float2(f01.z, f01.w), make_float2(f10.z, f10.w),
-                        make_float2(f11.z, f11.w), pp, oa[2 * g + 1], ob[2 * g + 1]);
-            }
-          } else {
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-              const int chunk = hsel * 4 + hh * 2 + g;
-              const uint4 u00 = *reinterpret_cast<const uint4*>(swz(slab, pp.L00, chunk));
-              const uint4 u01 = *reinterpret_cast<const uint4*>(swz(slab, pp.L01, chunk));
-              const uint4 u10 = *reinterpret_cast<const uint4*>(swz(slab, pp.L10, chunk));
-              const uint4 u11 = *reinterpret_cast<const uint4*>(swz(slab, pp.L11, chunk));
-              lerp_pair(bf16lo_hi(u00.x), bf16lo_hi(u01.x), bf16lo_hi(u10.x), bf16lo_hi(u11.x), pp,
-                        oa[4 * g + 0], ob[4 * g + 0]);
-              lerp_pair(bf16lo_hi(u00.y), bf16lo_hi(u01.y), bf16lo_hi(u10.y), bf16lo_hi(u11.y), pp,
-                        oa[4 * g + 1], ob[4 * g + 1]);
-              lerp_pair(bf16lo_hi(u00.z), bf16lo_hi(u01.z), bf16lo_hi(u10.z), bf16lo_hi(u11.z), pp,
-                        oa[4 * g + 2], ob[4 * g + 2]);
-              lerp_pair(bf16lo_hi(u00.w), bf16lo_hi(u01.w), bf16lo_hi(u10.w), bf16lo_hi(u11.w), pp,
-                        oa[4 * g + 3], ob[4 * g + 3]);
-            }
+          for (int gg = 0; gg < 2; ++gg) {
+            const uint32_t g16 = static_cast<uint32_t>(gg * 4 + cq) << 4;     // 4 channels: 4cq (+16)
+            const float4 f00 = ld_shared_f4((st + loff[0]) | (g16 ^ lxs[0]));
+            const float4 f01 = ld_shared_f4((st + loff[1]) | (g16 ^ lxs[1]));
+            const float4 f10 = ld_shared_f4((st + loff[2]) | (g16 ^ lxs[2]));
+            const float4 f11 = ld_shared_f4((st + loff[3]) | (g16 ^ lxs[3]));
+            lerp_column(make_float2(f00.x, f00.y), make_float2(f01.x, f01.y), make_float2(f10.x, f10.y),
+                        make_float2(f11.x, f11.y), cg, o[2 * gg]);
+            lerp_column(make_float2(f00.z, f00.w), make_float2(f01.z, f01.w), make_float2(f10.z, f10.w),
+                        make_float2(f11.z, f11.w), cg, o[2 * gg + 1]);
           }
-          tmem_st_32x32b_x8(acol + hh * 8, oa);
-          tmem_st_32x32b_x8(acol + 32 + hh * 8, ob);
+        } else {
+#pragma unroll
+          for (int gg = 0; gg < 2; ++gg) {
+            // 4 bf16 channels = half of a 16-byte chunk of the 64-channel line
+            const uint32_t g8 = ((static_cast<uint32_t>(hsel * 4 + gg * 2 + (cq >> 1)) << 4) ^ 0u);
+            const uint32_t h8 = static_cast<uint32_t>(cq & 1) << 3;
+            const uint2 u00 = ld_shared_u2(((st + loff[0]) | (g8 ^ lxs[0])) + h8);
+            const uint2 u01 = ld_shared_u2(((st + loff[1]) | (g8 ^ lxs[1])) + h8);
+            const uint2 u10 = ld_shared_u2(((st + loff[2]) | (g8 ^ lxs[2])) + h8);
+            const uint2 u11 = ld_shared_u2(((st + loff[3]) | (g8 ^ lxs[3])) + h8);
+            lerp_column(bf16lo_hi(u00.x), bf16lo_hi(u01.x), bf16lo_hi(u10.x), bf16lo_hi(u11.x), cg, o[2 * gg]);
+            lerp_column(bf16lo_hi(u00.y), bf16lo_hi(u01.y), bf16lo_hi(u10.y), bf16lo_hi(u11.y), cg, o[2 * gg + 1]);
+          }
         }
+        const uint32_t acol = tmem + kColA + s * 32 + hsel * 16;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          // lanes (jx, jx + 8) of the 16-lane half hf = rows 2 hf, 2 hf + 1
+          const uint32_t r[8] = {o[0][2 * hf], o[1][2 * hf], o[0][2 * hf + 1], o[1][2 * hf + 1],
+                                 o[2][2 * hf], o[3][2 * hf], o[2][2 * hf + 1], o[3][2 * hf + 1]};
+          tmem_st_16x256b_x2(acol + (static_cast<uint32_t>(32 * q + 16 * hf) << 16), r);
+        }
+        if (lane == 0 && warp == kWarpProd0) GKD_TR(7, it);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0 && !(skip_first && it == 0)) mbar_arrive(&ctl->afull[s]);
+        if (lane == 0 && warp == kWarpProd0) GKD_TR(8, it);
       }
     }
     tmem_wait_st();
@@ -559,10 +643,21 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
 
 }  // namespace tc
 
-static bool encode(EncodeTiledFn enc, CUtensorMap* m, CUtensorMapDataType dt, const void* base,
+#ifdef GKD_TRACE
+extern "C" __attribute__((visibility("default"))) int gkd_trace_read(void* host, int clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(host, tc::g_trace, sizeof(tc::g_trace));
+  if (e == cudaSuccess && clear) {
+    static unsigned long long zero[16][2048];
+    e = cudaMemcpyToSymbol(tc::g_trace, zero, sizeof(zero));
+  }
+  return static_cast<int>(e);
+}
+#endif
+
+static bool encode(EncodeTiledFn enc, CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
                    const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
-  const cuuint32_t es[4] = {1, 1, 1, 1};
-  CUresult r = enc(m, dt, 4, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, dt, rank, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -577,19 +672,30 @@ cudaError_t launch_heatmap_tc(HeatmapTcArgs& a, const void* feat, const void* ke
     return cudaErrorNotSupported;
   }
   const cuuint64_t C = a.C, w = a.w, h = a.h, B = a.B;
+  a.feat_5d = 0;
   if (a.feat_bf16) {
     const cuuint64_t dims[4] = {C, w, h, B};
     const cuuint64_t strides[3] = {C * 2, w * C * 2, h * w * C * 2};
     const cuuint32_t box[4] = {64, tc::kSlabCols, tc::kSlabRows, 1};
-    if (!encode(enc, &a.tmap_feat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, feat, dims, strides, box)) {
+    if (!encode(enc, &a.tmap_feat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, feat, dims, strides, box)) {
       *why = "tensor map encoding failed for the bf16 feature map";
       return cudaErrorInvalidValue;
     }
+  } else if (a.C % 32 == 0) {
+    // channels split as (32, C/32) so one box brings both 32-channel halves of a chunk
+    const cuuint64_t dims[5] = {32, w, h, C / 32, B};
+    const cuuint64_t strides[4] = {C * 4, w * C * 4, 128, h * w * C * 4};
+    const cuuint32_t box[5] = {32, tc::kSlabCols, tc::kSlabRows, 2, 1};
+    if (!encode(enc, &a.tmap_feat, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, feat, dims, strides, box)) {
+      *why = "tensor map encoding failed for the fp32 feature map";
+      return cudaErrorInvalidValue;
+    }
+    a.feat_5d = 1;
   } else {
     const cuuint64_t dims[4] = {C, w, h, B};
     const cuuint64_t strides[3] = {C * 4, w * C * 4, h * w * C * 4};
     const cuuint32_t box[4] = {32, tc::kSlabCols, tc::kSlabRows, 1};
-    if (!encode(enc, &a.tmap_feat, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, feat, dims, strides, box)) {
+    if (!encode(enc, &a.tmap_feat, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, feat, dims, strides, box)) {
       *why = "tensor map encoding failed for the fp32 feature map";
       return cudaErrorInvalidValue;
     }
@@ -600,12 +706,12 @@ cudaError_t launch_heatmap_tc(HeatmapTcArgs& a, const void* feat, const void* ke
     const cuuint64_t bstride = a.kern_shared ? M * K * C * 2 : static_cast<cuuint64_t>(kern_batch_stride) * 2;
     const cuuint64_t dims[4] = {C, K, M, Bk};
     const cuuint64_t strides[3] = {C * 2, K * C * 2, bstride};
-    const cuuint32_t box8[4] = {64, 8, 1, 1};
-    const cuuint32_t box32[4] = {64, 32, 1, 1};
-    if (!encode(enc, &a.tmap_kern8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kern, dims, strides, box8) ||
-        !encode(enc, &a.tmap_kern32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kern, dims, strides, box32)) {
-      *why = "tensor map encoding failed for the kernel rows";
-      return cudaErrorInvalidValue;
+    for (int i = 0; i < kKernMaps; ++i) {
+      const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(8 * (i + 1)), 1, 1};
+      if (!encode(enc, &a.tmap_kern[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, kern, dims, strides, box)) {
+        *why = "tensor map encoding failed for the kernel rows";
+        return cudaErrorInvalidValue;
+      }
     }
   }
   cudaError_t e = cudaFuncSetAttribute(tc::heatmap_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
