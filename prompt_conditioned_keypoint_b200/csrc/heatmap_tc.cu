@@ -42,14 +42,18 @@ __device__ unsigned long long g_trace[16][2048];
 #define GKD_TR(kind, idx) do { } while (0)
 #endif
 
-constexpr int kStages = 6;                       // ring: slab + kernel rows (smem), A operand (tmem)
-constexpr int kChunk = 64;                       // channels per K-chunk
+constexpr int kStages = 3;                       // ring: slab + kernel rows (smem), A operand (tmem)
+constexpr int kChunk = 128;                      // channels per stage: two 64-channel sub-chunks
+constexpr int kSub = 64;                         // channels per A sub-chunk (32 TMEM columns)
 constexpr int kMaxN = 160;                       // accumulator columns per tile
 constexpr int kUnitRows = 4, kUnitCols = 32;     // one M=128 tile: 4 output rows x 32 output columns
 constexpr int kSlabRows = 2, kSlabCols = 10, kSlabLines = kSlabRows * kSlabCols;
-constexpr int kSlabBytes = 8192;                 // fp32: two halves (at 0 and 2560, or 0 and 4096); bf16: one
-constexpr int kBBytes = kMaxN * 128;
-constexpr int kStageBytes = kSlabBytes + kBBytes;  // 28 KB, 1 KB aligned
+constexpr int kPlaneBytes = kSlabLines * 128;    // one 128-byte-wide slab plane (32 fp32 / 64 bf16 channels)
+constexpr int kPlaneSplit = 3072;                // plane pitch when each plane is its own box (1 KB aligned)
+constexpr int kSlabBytes = 4 * kPlaneSplit;      // fp32: 4 planes; bf16: 2 planes
+constexpr int kBSubBytes = kMaxN * 128;          // kernel rows of one sub-chunk
+constexpr int kBBytes = 2 * kBSubBytes;
+constexpr int kStageBytes = kSlabBytes + kBBytes;  // 52 KB, 1 KB aligned
 constexpr int kEpiCols = 16;                     // accumulator columns per epilogue group
 constexpr int kEpiStride = 40;                   // floats per (column, row) line of the epilogue tile
 constexpr int kEpiBufBytes = kEpiCols * kUnitRows * kEpiStride * 4;   // 10 KB
@@ -58,7 +62,7 @@ constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kWarpProd0 = 6;
 constexpr int kNumProdWarps = 8, kNumEpiWarps = 4;
 constexpr int kEpiBarrier = 1;                   // named barrier of the four epilogue warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColA = 2 * kMaxN;            // accumulators at 0 and 160; A stages at 320 + 32 s
+constexpr uint32_t kColA = 2 * kMaxN;            // accumulators at 0 and 160; A stages at 320 + 64 s
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 2 * kEpiBufBytes + 512;
 
 struct Smem {            // control block placed after the stage and epilogue buffers
@@ -365,45 +369,49 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
 
   if (warp == kWarpTma) {
     // ---------------------------------------------------------------- TMA
-    uint32_t it = 0;
+    uint32_t it = 0, st = 0, ph = 0;            // stage index / its use parity
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
-    const uint32_t slab_bytes = (a.feat_bf16 ? 1 : 2) * kSlabLines * 128;
+    const uint32_t slab_bytes = (a.feat_bf16 ? 2 : 4) * kPlaneBytes;
+    const int nplanes = a.feat_bf16 ? 2 : 4, plane_ch = a.feat_bf16 ? 64 : 32;
     for (unsigned long long u = ubeg; u < uend && ok; ++u) {
       const int b = static_cast<int>(u / nU), j = static_cast<int>(u % nU);
       if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
       if (ci.n == 0) continue;
       const int vb = j / ncb, ub = j % ncb;
       const int bk = a.kern_shared ? 0 : b;
+      const uint32_t bytes = slab_bytes + 2 * (ci.len0 + ci.len1) * 128;
+      const CUtensorMap* km0 = ci.len0 ? &a.tmap_kern[(ci.len0 >> 3) - 1] : nullptr;
+      const CUtensorMap* km1 = ci.len1 ? &a.tmap_kern[(ci.len1 >> 3) - 1] : nullptr;
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
-        const int s = it % kStages;
-        const uint32_t use = it / kStages;
-        if (use > 0 && !mbar_wait_bounded(&ctl->empty[s], (use & 1) ^ 1, lim, abortp)) {
+        if (it >= kStages && !mbar_wait_bounded(&ctl->empty[st], ph ^ 1, lim, abortp)) {
           if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
           ok = false;
           break;
         }
         if (lane == 0) {
           GKD_TR(0, it);
-          uint8_t* st = smem + s * kStageBytes;
-          mbar_arrive_expect_tx(&ctl->full[s], slab_bytes + (ci.len0 + ci.len1) * 128);
+          uint8_t* sp = smem + st * kStageBytes;
+          uint64_t* fb = &ctl->full[st];
+          mbar_arrive_expect_tx(fb, bytes);
           const int c0 = ch * kChunk;
-          if (a.feat_bf16) {
-            tma_load_4d(st, &a.tmap_feat, &ctl->full[s], c0, 8 * ub - 1, vb - 1, b);
-          } else if (a.feat_5d) {
-            tma_load_5d(st, &a.tmap_feat, &ctl->full[s], 0, 8 * ub - 1, vb - 1, c0 / 32, b);
+          if (a.feat_5d) {
+            tma_load_5d(sp, &a.tmap_feat, fb, 0, 8 * ub - 1, vb - 1, c0 / plane_ch, b);
           } else {
-            tma_load_4d(st, &a.tmap_feat, &ctl->full[s], c0, 8 * ub - 1, vb - 1, b);
-            tma_load_4d(st + 4096, &a.tmap_feat, &ctl->full[s], c0 + 32, 8 * ub - 1, vb - 1, b);
+            for (int p = 0; p < nplanes; ++p)
+              tma_load_4d(sp + p * kPlaneSplit, &a.tmap_feat, fb, c0 + p * plane_ch, 8 * ub - 1, vb - 1, b);
           }
-          uint8_t* bdst = st + kSlabBytes;
-          if (ci.len0) tma_load_4d(bdst, &a.tmap_kern[(ci.len0 >> 3) - 1], &ctl->full[s], c0, ci.kmin0, 0, bk);
-          if (ci.len1)
-            tma_load_4d(bdst + ci.off1 * 128, &a.tmap_kern[(ci.len1 >> 3) - 1], &ctl->full[s], c0, ci.kmin1, 1, bk);
+#pragma unroll
+          for (int hs = 0; hs < 2; ++hs) {
+            uint8_t* bdst = sp + kSlabBytes + hs * kBSubBytes;
+            if (km0) tma_load_4d(bdst, km0, fb, c0 + hs * kSub, ci.kmin0, 0, bk);
+            if (km1) tma_load_4d(bdst + ci.off1 * 128, km1, fb, c0 + hs * kSub, ci.kmin1, 1, bk);
+          }
           GKD_TR(1, it);
         }
         __syncwarp();
+        if (++st == kStages) { st = 0; ph ^= 1; }
       }
     }
     // drain: no load issued by this warp may still be landing in shared memory
@@ -416,7 +424,8 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     __syncwarp();
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA
-    uint32_t it = 0, v = 0;
+    uint32_t it = 0, v = 0, st = 0, ph = 0;
+    const uint64_t bdesc0 = make_bdesc(smem_base + kSlabBytes);
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
@@ -435,12 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       if (lane == 0) GKD_TR(13, v);
       tc_fence_after();
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
-        const int s = it % kStages;
-        const uint32_t par = (it / kStages) & 1;
         if (lane == 0) GKD_TR(4, it);
-        const bool okf = mbar_wait_bounded(&ctl->full[s], par, lim, abortp);
+        const bool okf = mbar_wait_bounded(&ctl->full[st], ph, lim, abortp);
         if (lane == 0) GKD_TR(5, it);
-        if (!okf || !mbar_wait_bounded(&ctl->afull[s], par, lim, abortp)) {
+        if (!okf || !mbar_wait_bounded(&ctl->afull[st], ph, lim, abortp)) {
           if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
           ok = false;
           break;
@@ -449,18 +456,23 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
         tc_fence_after();
         if (lane == 0) {
           GKD_TR(2, it);
-          const uint32_t bbase = smem_base + s * kStageBytes + kSlabBytes;
-          const uint32_t acol = tmem + kColA + s * 32;
+          const uint64_t bd = bdesc0 + ((st * kStageBytes) >> 4);
+          const uint32_t acol = tmem + kColA + st * 64;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            umma_ts_f16(dcol, acol + kk * 8, make_bdesc(bbase + kk * 32), idesc, (ch > 0 || kk > 0) ? 1u : 0u);
-            if (kk == 0) GKD_TR(12, it);
+          for (int hs = 0; hs < 2; ++hs) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              umma_ts_f16(dcol, acol + hs * 32 + kk * 8, bd + ((hs * kBSubBytes + kk * 32) >> 4), idesc,
+                          (ch > 0 || hs > 0 || kk > 0) ? 1u : 0u);
+              if (hs == 0 && kk == 0) GKD_TR(12, it);
+            }
           }
           GKD_TR(15, it);
-          umma_commit(&ctl->empty[s]);
+          umma_commit(&ctl->empty[st]);
           GKD_TR(3, it);
         }
         __syncwarp();
+        if (++st == kStages) { st = 0; ph ^= 1; }
       }
       if (!ok) break;
       if (lane == 0) {
@@ -553,9 +565,9 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     const int hsel = (warp - kWarpProd0) >> 2;   // which 32 channels of each chunk
     const int jx = lane >> 2, cq = lane & 3;      // column within the quadrant, channel quarter
     const bool skip_first = (a.debug_flags & kDbgSkipProducerArrive) != 0;
-    // line offset of this thread's channel half within a stage's slab
-    const int half_lines = a.feat_bf16 ? 0 : (a.feat_5d ? kSlabLines : 32);
-    uint32_t it = 0;
+    // slab plane pitch (in 128-byte lines) and the plane of each sub-chunk's channels
+    const int plane_lines = a.feat_5d ? kSlabLines : kPlaneSplit / 128;
+    uint32_t it = 0, st = 0, ph = 0;
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
@@ -564,69 +576,75 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
       if (ci.n == 0) continue;
       const Column4 cg = column_geometry(a, j / ncb, j % ncb, q, jx);
-      // per tap: byte offset of its line inside a stage, and its swizzle pattern
-      uint32_t loff[4], lxs[4];
+      // per tap and sub-chunk: byte offset of its line inside a stage, and its swizzle pattern
+      uint32_t loff[2][4], lxs[2][4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int line = hsel * half_lines + cg.L[k];
-        loff[k] = static_cast<uint32_t>(line) * 128u;
-        lxs[k] = static_cast<uint32_t>(line & 7) << 4;
+      for (int hs = 0; hs < 2; ++hs) {
+        const int plane = a.feat_bf16 ? hs : 2 * hs + hsel;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int line = plane * plane_lines + cg.L[k];
+          loff[hs][k] = static_cast<uint32_t>(line) * 128u;
+          lxs[hs][k] = static_cast<uint32_t>(line & 7) << 4;
+        }
       }
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
-        const int s = it % kStages;
-        const uint32_t use = it / kStages;
-        if (!mbar_wait_bounded(&ctl->full[s], use & 1, lim, abortp) ||
-            (use > 0 && !mbar_wait_bounded(&ctl->empty[s], (use & 1) ^ 1, lim, abortp))) {
+        if (!mbar_wait_bounded(&ctl->full[st], ph, lim, abortp) ||
+            (it >= kStages && !mbar_wait_bounded(&ctl->empty[st], ph ^ 1, lim, abortp))) {
           if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0 && warp == kWarpProd0) GKD_TR(6, it);
-        const uint32_t st = smem_base + s * kStageBytes;
-        // o[p][r]: channel pair p (4cq, 4cq+2, 16+4cq, 18+4cq of this warp's 32 channels), row r
-        uint32_t o[4][4];
-        if (!a.feat_bf16) {
+        const uint32_t sp = smem_base + st * kStageBytes;
 #pragma unroll
-          for (int gg = 0; gg < 2; ++gg) {
-            const uint32_t g16 = static_cast<uint32_t>(gg * 4 + cq) << 4;     // 4 channels: 4cq (+16)
-            const float4 f00 = ld_shared_f4((st + loff[0]) | (g16 ^ lxs[0]));
-            const float4 f01 = ld_shared_f4((st + loff[1]) | (g16 ^ lxs[1]));
-            const float4 f10 = ld_shared_f4((st + loff[2]) | (g16 ^ lxs[2]));
-            const float4 f11 = ld_shared_f4((st + loff[3]) | (g16 ^ lxs[3]));
-            lerp_column(make_float2(f00.x, f00.y), make_float2(f01.x, f01.y), make_float2(f10.x, f10.y),
-                        make_float2(f11.x, f11.y), cg, o[2 * gg]);
-            lerp_column(make_float2(f00.z, f00.w), make_float2(f01.z, f01.w), make_float2(f10.z, f10.w),
-                        make_float2(f11.z, f11.w), cg, o[2 * gg + 1]);
+        for (int hs = 0; hs < 2; ++hs) {
+          // o[p][r]: channel pair p (4cq, 4cq+2, 16+4cq, 18+4cq of this warp's 32 channels), row r
+          uint32_t o[4][4];
+          if (!a.feat_bf16) {
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg) {
+              const uint32_t g16 = static_cast<uint32_t>(gg * 4 + cq) << 4;     // 4 channels: 4cq (+16)
+              const float4 f00 = ld_shared_f4((sp + loff[hs][0]) | (g16 ^ lxs[hs][0]));
+              const float4 f01 = ld_shared_f4((sp + loff[hs][1]) | (g16 ^ lxs[hs][1]));
+              const float4 f10 = ld_shared_f4((sp + loff[hs][2]) | (g16 ^ lxs[hs][2]));
+              const float4 f11 = ld_shared_f4((sp + loff[hs][3]) | (g16 ^ lxs[hs][3]));
+              lerp_column(make_float2(f00.x, f00.y), make_float2(f01.x, f01.y), make_float2(f10.x, f10.y),
+                          make_float2(f11.x, f11.y), cg, o[2 * gg]);
+              lerp_column(make_float2(f00.z, f00.w), make_float2(f01.z, f01.w), make_float2(f10.z, f10.w),
+                          make_float2(f11.z, f11.w), cg, o[2 * gg + 1]);
+            }
+          } else {
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg) {
+              // 4 bf16 channels = half of a 16-byte chunk of the 64-channel line
+              const uint32_t g8 = static_cast<uint32_t>(hsel * 4 + gg * 2 + (cq >> 1)) << 4;
+              const uint32_t h8 = static_cast<uint32_t>(cq & 1) << 3;
+              const uint2 u00 = ld_shared_u2(((sp + loff[hs][0]) | (g8 ^ lxs[hs][0])) + h8);
+              const uint2 u01 = ld_shared_u2(((sp + loff[hs][1]) | (g8 ^ lxs[hs][1])) + h8);
+              const uint2 u10 = ld_shared_u2(((sp + loff[hs][2]) | (g8 ^ lxs[hs][2])) + h8);
+              const uint2 u11 = ld_shared_u2(((sp + loff[hs][3]) | (g8 ^ lxs[hs][3])) + h8);
+              lerp_column(bf16lo_hi(u00.x), bf16lo_hi(u01.x), bf16lo_hi(u10.x), bf16lo_hi(u11.x), cg, o[2 * gg]);
+              lerp_column(bf16lo_hi(u00.y), bf16lo_hi(u01.y), bf16lo_hi(u10.y), bf16lo_hi(u11.y), cg, o[2 * gg + 1]);
+            }
           }
-        } else {
+          const uint32_t acol = tmem + kColA + st * 64 + hs * 32 + hsel * 16;
 #pragma unroll
-          for (int gg = 0; gg < 2; ++gg) {
-            // 4 bf16 channels = half of a 16-byte chunk of the 64-channel line
-            const uint32_t g8 = ((static_cast<uint32_t>(hsel * 4 + gg * 2 + (cq >> 1)) << 4) ^ 0u);
-            const uint32_t h8 = static_cast<uint32_t>(cq & 1) << 3;
-            const uint2 u00 = ld_shared_u2(((st + loff[0]) | (g8 ^ lxs[0])) + h8);
-            const uint2 u01 = ld_shared_u2(((st + loff[1]) | (g8 ^ lxs[1])) + h8);
-            const uint2 u10 = ld_shared_u2(((st + loff[2]) | (g8 ^ lxs[2])) + h8);
-            const uint2 u11 = ld_shared_u2(((st + loff[3]) | (g8 ^ lxs[3])) + h8);
-            lerp_column(bf16lo_hi(u00.x), bf16lo_hi(u01.x), bf16lo_hi(u10.x), bf16lo_hi(u11.x), cg, o[2 * gg]);
-            lerp_column(bf16lo_hi(u00.y), bf16lo_hi(u01.y), bf16lo_hi(u10.y), bf16lo_hi(u11.y), cg, o[2 * gg + 1]);
+          for (int hf = 0; hf < 2; ++hf) {
+            // lanes (jx, jx + 8) of the 16-lane half hf = rows 2 hf, 2 hf + 1
+            const uint32_t r[8] = {o[0][2 * hf], o[1][2 * hf], o[0][2 * hf + 1], o[1][2 * hf + 1],
+                                   o[2][2 * hf], o[3][2 * hf], o[2][2 * hf + 1], o[3][2 * hf + 1]};
+            tmem_st_16x256b_x2(acol + (static_cast<uint32_t>(32 * q + 16 * hf) << 16), r);
           }
-        }
-        const uint32_t acol = tmem + kColA + s * 32 + hsel * 16;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          // lanes (jx, jx + 8) of the 16-lane half hf = rows 2 hf, 2 hf + 1
-          const uint32_t r[8] = {o[0][2 * hf], o[1][2 * hf], o[0][2 * hf + 1], o[1][2 * hf + 1],
-                                 o[2][2 * hf], o[3][2 * hf], o[2][2 * hf + 1], o[3][2 * hf + 1]};
-          tmem_st_16x256b_x2(acol + (static_cast<uint32_t>(32 * q + 16 * hf) << 16), r);
         }
         if (lane == 0 && warp == kWarpProd0) GKD_TR(7, it);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0 && !(skip_first && it == 0)) mbar_arrive(&ctl->afull[s]);
+        if (lane == 0 && !(skip_first && it == 0)) mbar_arrive(&ctl->afull[st]);
         if (lane == 0 && warp == kWarpProd0) GKD_TR(8, it);
+        if (++st == kStages) { st = 0; ph ^= 1; }
       }
     }
     tmem_wait_st();
@@ -673,30 +691,26 @@ cudaError_t launch_heatmap_tc(HeatmapTcArgs& a, const void* feat, const void* ke
   }
   const cuuint64_t C = a.C, w = a.w, h = a.h, B = a.B;
   a.feat_5d = 0;
-  if (a.feat_bf16) {
-    const cuuint64_t dims[4] = {C, w, h, B};
-    const cuuint64_t strides[3] = {C * 2, w * C * 2, h * w * C * 2};
-    const cuuint32_t box[4] = {64, tc::kSlabCols, tc::kSlabRows, 1};
-    if (!encode(enc, &a.tmap_feat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, feat, dims, strides, box)) {
-      *why = "tensor map encoding failed for the bf16 feature map";
-      return cudaErrorInvalidValue;
-    }
-  } else if (a.C % 32 == 0) {
-    // channels split as (32, C/32) so one box brings both 32-channel halves of a chunk
-    const cuuint64_t dims[5] = {32, w, h, C / 32, B};
-    const cuuint64_t strides[4] = {C * 4, w * C * 4, 128, h * w * C * 4};
-    const cuuint32_t box[5] = {32, tc::kSlabCols, tc::kSlabRows, 2, 1};
-    if (!encode(enc, &a.tmap_feat, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, feat, dims, strides, box)) {
-      *why = "tensor map encoding failed for the fp32 feature map";
+  const cuuint64_t elt = a.feat_bf16 ? 2 : 4;
+  const cuuint64_t plane_ch = a.feat_bf16 ? 64 : 32;       // channels of one 128-byte slab plane
+  const CUtensorMapDataType fdt = a.feat_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if (a.C % plane_ch == 0) {
+    // channels split as (plane, C / plane) so one box brings every plane of a 128-channel stage
+    const cuuint64_t dims[5] = {plane_ch, w, h, C / plane_ch, B};
+    const cuuint64_t strides[4] = {C * elt, w * C * elt, 128, h * w * C * elt};
+    const cuuint32_t box[5] = {static_cast<cuuint32_t>(plane_ch), tc::kSlabCols, tc::kSlabRows,
+                               static_cast<cuuint32_t>(tc::kChunk / plane_ch), 1};
+    if (!encode(enc, &a.tmap_feat, fdt, 5, feat, dims, strides, box)) {
+      *why = "tensor map encoding failed for the feature map";
       return cudaErrorInvalidValue;
     }
     a.feat_5d = 1;
   } else {
     const cuuint64_t dims[4] = {C, w, h, B};
-    const cuuint64_t strides[3] = {C * 4, w * C * 4, h * w * C * 4};
-    const cuuint32_t box[4] = {32, tc::kSlabCols, tc::kSlabRows, 1};
-    if (!encode(enc, &a.tmap_feat, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, feat, dims, strides, box)) {
-      *why = "tensor map encoding failed for the fp32 feature map";
+    const cuuint64_t strides[3] = {C * elt, w * C * elt, h * w * C * elt};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(plane_ch), tc::kSlabCols, tc::kSlabRows, 1};
+    if (!encode(enc, &a.tmap_feat, fdt, 4, feat, dims, strides, box)) {
+      *why = "tensor map encoding failed for the feature map";
       return cudaErrorInvalidValue;
     }
   }
