@@ -36,13 +36,15 @@ namespace tc {
 // at each hand-off between roles; read back with gkd_trace_read().
 #ifdef GKD_TRACE
 __device__ unsigned long long g_trace[16][2048];
+__device__ unsigned long long g_cta[1024][4];     // per CTA: start, end (ns), units, sum of n
 #define GKD_TR(kind, idx) \
   do { if (blockIdx.x == 0 && (idx) < 2048u) g_trace[kind][idx] = global_timer_ns(); } while (0)
 #else
 #define GKD_TR(kind, idx) do { } while (0)
 #endif
 
-constexpr int kStages = 3;                       // ring: slab + kernel rows (smem), A operand (tmem)
+constexpr int kSlabStages = 6;                   // slab ring (smem), freed by the producers
+constexpr int kStages = 3;                       // kernel rows (smem) + A operand (tmem), freed by the MMA
 constexpr int kChunk = 128;                      // channels per stage: two 64-channel sub-chunks
 constexpr int kSub = 64;                         // channels per A sub-chunk (32 TMEM columns)
 constexpr int kMaxN = 160;                       // accumulator columns per tile
@@ -52,22 +54,24 @@ constexpr int kPlaneBytes = kSlabLines * 128;    // one 128-byte-wide slab plane
 constexpr int kPlaneSplit = 3072;                // plane pitch when each plane is its own box (1 KB aligned)
 constexpr int kSlabBytes = 4 * kPlaneSplit;      // fp32: 4 planes; bf16: 2 planes
 constexpr int kBSubBytes = kMaxN * 128;          // kernel rows of one sub-chunk
-constexpr int kBBytes = 2 * kBSubBytes;
-constexpr int kStageBytes = kSlabBytes + kBBytes;  // 52 KB, 1 KB aligned
+constexpr int kBBytes = 2 * kBSubBytes;          // 40 KB per stage, 1 KB aligned
 constexpr int kEpiCols = 16;                     // accumulator columns per epilogue group
 constexpr int kEpiStride = 40;                   // floats per (column, row) line of the epilogue tile
 constexpr int kEpiBufBytes = kEpiCols * kUnitRows * kEpiStride * 4;   // 10 KB
-constexpr int kNumWarps = 14, kThreads = kNumWarps * 32;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kWarpProd0 = 6;
-constexpr int kNumProdWarps = 8, kNumEpiWarps = 4;
+constexpr int kNumProdWarps = 16, kNumEpiWarps = 4;
+constexpr int kNumWarps = 3 + kNumEpiWarps + kNumProdWarps, kThreads = kNumWarps * 32;
+constexpr int kWarpTma = 0, kWarpTmaB = 1, kWarpMma = 2, kWarpEpi0 = 3, kWarpProd0 = 3 + kNumEpiWarps;
 constexpr int kEpiBarrier = 1;                   // named barrier of the four epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColA = 2 * kMaxN;            // accumulators at 0 and 160; A stages at 320 + 64 s
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 2 * kEpiBufBytes + 512;
+constexpr size_t kSmemBytes =
+    1024 + static_cast<size_t>(kSlabStages) * kSlabBytes + static_cast<size_t>(kStages) * kBBytes + 2 * kEpiBufBytes + 512;
 
 struct Smem {            // control block placed after the stage and epilogue buffers
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t sfull[kSlabStages];
+  uint64_t sempty[kSlabStages];
+  uint64_t full[kStages];      // kernel rows landed
+  uint64_t empty[kStages];     // MMA done with kernel rows and A operand
   uint64_t afull[kStages];
   uint64_t accfull[2];
   uint64_t accempty[2];
@@ -150,10 +154,9 @@ __device__ __forceinline__ int crop_n_serial(const HeatmapTcArgs& a, int b) {
   return (off + 15) & ~15;
 }
 
-// Relative cost of one unit with n accumulator columns: the slowest of the
-// upsample producers (independent of n), the kernel-row copy (grows with n)
-// and the MMAs.
-__device__ __forceinline__ long long unit_cost(int n) { return n == 0 ? 0 : max(2 * n + 80, 230); }
+// Relative cost of one unit with n accumulator columns (measured on B200: a unit
+// costs about 6 us plus about 0.01 us per accumulator column).
+__device__ __forceinline__ long long unit_cost(int n) { return n == 0 ? 0 : n + 640; }
 
 __device__ __forceinline__ void src_taps(int d, int n, int& i0, int& i1, float& lam) {
   const float s = fmaxf((static_cast<float>(d) + 0.5f) * 0.25f - 0.5f, 0.0f);
@@ -261,7 +264,8 @@ __device__ __forceinline__ void st_shared_f32(uint32_t addr, uint32_t v) {
 __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_constant__ HeatmapTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* epi_buf = smem + kStages * kStageBytes;
+  uint8_t* bring = smem + kSlabStages * kSlabBytes;          // kernel-row stages
+  uint8_t* epi_buf = bring + kStages * kBBytes;
   Smem* ctl = reinterpret_cast<Smem*>(epi_buf + 2 * kEpiBufBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
@@ -275,6 +279,10 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
 
   // ---------------- prologue: barriers, TMEM, work partition ----------------
   if (tid == 0) {
+    for (int s = 0; s < kSlabStages; ++s) {
+      mbar_init(&ctl->sfull[s], 1);
+      mbar_init(&ctl->sempty[s], kNumProdWarps);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
@@ -295,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     tmem_alloc(&ctl->tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kWarpTma && lane < 1 + kKernMaps) {
+  if (warp == kWarpTmaB && lane < 1 + kKernMaps) {
     tma_prefetch_desc(lane == 0 ? &a.tmap_feat : &a.tmap_kern[lane - 1]);
   }
   __syncthreads();
@@ -363,13 +371,16 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   const unsigned long long ubeg = ctl->unit_begin, uend = ctl->unit_end;
+#ifdef GKD_TRACE
+  if (tid == 0 && blockIdx.x < 1024) g_cta[blockIdx.x][0] = global_timer_ns();
+#endif
   const uint64_t lim = a.wait_limit_ns;
   volatile int* abortp = &ctl->abort_flag;
   const uint32_t smem_base = smem_u32(smem);
 
   if (warp == kWarpTma) {
-    // ---------------------------------------------------------------- TMA
-    uint32_t it = 0, st = 0, ph = 0;            // stage index / its use parity
+    // ---------------------------------------------------------------- TMA: feature slabs
+    uint32_t it = 0, st = 0, ph = 0;
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
@@ -380,8 +391,51 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
       if (ci.n == 0) continue;
       const int vb = j / ncb, ub = j % ncb;
+      for (int ch = 0; ch < nchunks; ++ch, ++it) {
+        if (it >= kSlabStages && !mbar_wait_bounded(&ctl->sempty[st], ph ^ 1, lim, abortp)) {
+          if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          GKD_TR(0, it);
+          uint8_t* sp = smem + st * kSlabBytes;
+          uint64_t* fb = &ctl->sfull[st];
+          mbar_arrive_expect_tx(fb, slab_bytes);
+          const int c0 = ch * kChunk;
+          if (a.feat_5d) {
+            tma_load_5d(sp, &a.tmap_feat, fb, 0, 8 * ub - 1, vb - 1, c0 / plane_ch, b);
+          } else {
+            for (int p = 0; p < nplanes; ++p)
+              tma_load_4d(sp + p * kPlaneSplit, &a.tmap_feat, fb, c0 + p * plane_ch, 8 * ub - 1, vb - 1, b);
+          }
+          GKD_TR(1, it);
+        }
+        __syncwarp();
+        if (++st == kSlabStages) { st = 0; ph ^= 1; }
+      }
+    }
+    // drain: no load issued by this warp may still be landing in shared memory
+    if (lane == 0) {
+      for (uint32_t k = 0; k < kSlabStages && k < it; ++k) {
+        const uint32_t last = it - 1 - k;
+        if (!mbar_wait_drain(&ctl->sfull[last % kSlabStages], (last / kSlabStages) & 1, lim))
+          atomicOr(a.err, kErrTimeout);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kWarpTmaB) {
+    // ---------------------------------------------------------------- TMA: kernel rows (B operand)
+    uint32_t it = 0, st = 0, ph = 0;
+    int cur_b = -1;
+    CropInfo ci{};
+    bool ok = true;
+    for (unsigned long long u = ubeg; u < uend && ok; ++u) {
+      const int b = static_cast<int>(u / nU);
+      if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
+      if (ci.n == 0) continue;
       const int bk = a.kern_shared ? 0 : b;
-      const uint32_t bytes = slab_bytes + 2 * (ci.len0 + ci.len1) * 128;
+      const uint32_t bytes = 2 * (ci.len0 + ci.len1) * 128;
       const CUtensorMap* km0 = ci.len0 ? &a.tmap_kern[(ci.len0 >> 3) - 1] : nullptr;
       const CUtensorMap* km1 = ci.len1 ? &a.tmap_kern[(ci.len1 >> 3) - 1] : nullptr;
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
@@ -391,30 +445,21 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
           break;
         }
         if (lane == 0) {
-          GKD_TR(0, it);
-          uint8_t* sp = smem + st * kStageBytes;
+          uint8_t* bp = bring + st * kBBytes;
           uint64_t* fb = &ctl->full[st];
           mbar_arrive_expect_tx(fb, bytes);
           const int c0 = ch * kChunk;
-          if (a.feat_5d) {
-            tma_load_5d(sp, &a.tmap_feat, fb, 0, 8 * ub - 1, vb - 1, c0 / plane_ch, b);
-          } else {
-            for (int p = 0; p < nplanes; ++p)
-              tma_load_4d(sp + p * kPlaneSplit, &a.tmap_feat, fb, c0 + p * plane_ch, 8 * ub - 1, vb - 1, b);
-          }
 #pragma unroll
           for (int hs = 0; hs < 2; ++hs) {
-            uint8_t* bdst = sp + kSlabBytes + hs * kBSubBytes;
+            uint8_t* bdst = bp + hs * kBSubBytes;
             if (km0) tma_load_4d(bdst, km0, fb, c0 + hs * kSub, ci.kmin0, 0, bk);
             if (km1) tma_load_4d(bdst + ci.off1 * 128, km1, fb, c0 + hs * kSub, ci.kmin1, 1, bk);
           }
-          GKD_TR(1, it);
         }
         __syncwarp();
         if (++st == kStages) { st = 0; ph ^= 1; }
       }
     }
-    // drain: no load issued by this warp may still be landing in shared memory
     if (lane == 0) {
       for (uint32_t k = 0; k < kStages && k < it; ++k) {
         const uint32_t last = it - 1 - k;
@@ -425,7 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA
     uint32_t it = 0, v = 0, st = 0, ph = 0;
-    const uint64_t bdesc0 = make_bdesc(smem_base + kSlabBytes);
+#ifdef GKD_TRACE
+    unsigned long long trace_sum_n = 0;
+#endif
+    const uint64_t bdesc0 = make_bdesc(smem_u32(bring));
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
@@ -434,6 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
       if (ci.n == 0) continue;
       const uint32_t idesc = make_idesc(ci.n);
+#ifdef GKD_TRACE
+      trace_sum_n += ci.n;
+#endif
       const int buf = v & 1;
       const uint32_t dcol = tmem + buf * kMaxN;
       if (v >= 2 && !mbar_wait_bounded(&ctl->accempty[buf], ((v >> 1) & 1) ^ 1, lim, abortp)) {
@@ -456,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
         tc_fence_after();
         if (lane == 0) {
           GKD_TR(2, it);
-          const uint64_t bd = bdesc0 + ((st * kStageBytes) >> 4);
+          const uint64_t bd = bdesc0 + ((st * kBBytes) >> 4);
           const uint32_t acol = tmem + kColA + st * 64;
 #pragma unroll
           for (int hs = 0; hs < 2; ++hs) {
@@ -487,6 +538,13 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       umma_commit(&ctl->drain);
       if (!mbar_wait_drain(&ctl->drain, 0, lim)) atomicOr(a.err, kErrTimeout);
     }
+#ifdef GKD_TRACE
+    if (lane == 0 && blockIdx.x < 1024) {
+      g_cta[blockIdx.x][1] = global_timer_ns();
+      g_cta[blockIdx.x][2] = v;
+      g_cta[blockIdx.x][3] = trace_sum_n;
+    }
+#endif
     __syncwarp();
   } else if (warp < kWarpProd0) {
     // ---------------------------------------------------------------- epilogue
@@ -562,12 +620,17 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   } else {
     // ---------------------------------------------------------------- upsample producers
     const int q = warp & 3;
-    const int hsel = (warp - kWarpProd0) >> 2;   // which 32 channels of each chunk
-    const int jx = lane >> 2, cq = lane & 3;      // column within the quadrant, channel quarter
+    const int quarter = (warp - kWarpProd0) >> 2;  // which 16 channels of each 64-channel sub-chunk
+    const int jx = lane >> 2, cq = lane & 3;       // column within the quadrant, 4-channel group
     const bool skip_first = (a.debug_flags & kDbgSkipProducerArrive) != 0;
-    // slab plane pitch (in 128-byte lines) and the plane of each sub-chunk's channels
+    // slab plane pitch (in 128-byte lines)
     const int plane_lines = a.feat_5d ? kSlabLines : kPlaneSplit / 128;
-    uint32_t it = 0, st = 0, ph = 0;
+    // this thread's 4 channels inside its plane line: fp32 planes are 32 channels
+    // (16-byte chunk = 4 channels), bf16 planes 64 channels (8-byte half of a chunk)
+    const uint32_t g16 = a.feat_bf16 ? static_cast<uint32_t>(2 * quarter + (cq >> 1)) << 4
+                                     : static_cast<uint32_t>(4 * (quarter & 1) + cq) << 4;
+    const uint32_t h8 = a.feat_bf16 ? static_cast<uint32_t>(cq & 1) << 3 : 0u;
+    uint32_t it = 0, st = 0, ph = 0, ss = 0, sph = 0;   // A-ring and slab-ring positions
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
@@ -576,20 +639,19 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
       if (ci.n == 0) continue;
       const Column4 cg = column_geometry(a, j / ncb, j % ncb, q, jx);
-      // per tap and sub-chunk: byte offset of its line inside a stage, and its swizzle pattern
-      uint32_t loff[2][4], lxs[2][4];
+      // per tap and sub-chunk: byte address offset of this thread's 4 channels inside a stage
+      uint32_t toff[2][4];
 #pragma unroll
       for (int hs = 0; hs < 2; ++hs) {
-        const int plane = a.feat_bf16 ? hs : 2 * hs + hsel;
+        const int plane = a.feat_bf16 ? hs : 2 * hs + (quarter >> 1);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int line = plane * plane_lines + cg.L[k];
-          loff[hs][k] = static_cast<uint32_t>(line) * 128u;
-          lxs[hs][k] = static_cast<uint32_t>(line & 7) << 4;
+          toff[hs][k] = (static_cast<uint32_t>(line) * 128u | (g16 ^ (static_cast<uint32_t>(line & 7) << 4))) + h8;
         }
       }
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
-        if (!mbar_wait_bounded(&ctl->full[st], ph, lim, abortp) ||
+        if (!mbar_wait_bounded(&ctl->sfull[ss], sph, lim, abortp) ||
             (it >= kStages && !mbar_wait_bounded(&ctl->empty[st], ph ^ 1, lim, abortp))) {
           if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
           ok = false;
@@ -597,54 +659,47 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
         }
         tc_fence_after();
         if (lane == 0 && warp == kWarpProd0) GKD_TR(6, it);
-        const uint32_t sp = smem_base + st * kStageBytes;
+        const uint32_t sp = smem_base + ss * kSlabBytes;
 #pragma unroll
         for (int hs = 0; hs < 2; ++hs) {
-          // o[p][r]: channel pair p (4cq, 4cq+2, 16+4cq, 18+4cq of this warp's 32 channels), row r
-          uint32_t o[4][4];
+          // o[p][r]: channel pair p (4cq, 4cq+2 of this warp's 16 channels), row r
+          uint32_t o[2][4];
           if (!a.feat_bf16) {
-#pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-              const uint32_t g16 = static_cast<uint32_t>(gg * 4 + cq) << 4;     // 4 channels: 4cq (+16)
-              const float4 f00 = ld_shared_f4((sp + loff[hs][0]) | (g16 ^ lxs[hs][0]));
-              const float4 f01 = ld_shared_f4((sp + loff[hs][1]) | (g16 ^ lxs[hs][1]));
-              const float4 f10 = ld_shared_f4((sp + loff[hs][2]) | (g16 ^ lxs[hs][2]));
-              const float4 f11 = ld_shared_f4((sp + loff[hs][3]) | (g16 ^ lxs[hs][3]));
-              lerp_column(make_float2(f00.x, f00.y), make_float2(f01.x, f01.y), make_float2(f10.x, f10.y),
-                          make_float2(f11.x, f11.y), cg, o[2 * gg]);
-              lerp_column(make_float2(f00.z, f00.w), make_float2(f01.z, f01.w), make_float2(f10.z, f10.w),
-                          make_float2(f11.z, f11.w), cg, o[2 * gg + 1]);
-            }
+            const float4 f00 = ld_shared_f4(sp + toff[hs][0]);
+            const float4 f01 = ld_shared_f4(sp + toff[hs][1]);
+            const float4 f10 = ld_shared_f4(sp + toff[hs][2]);
+            const float4 f11 = ld_shared_f4(sp + toff[hs][3]);
+            lerp_column(make_float2(f00.x, f00.y), make_float2(f01.x, f01.y), make_float2(f10.x, f10.y),
+                        make_float2(f11.x, f11.y), cg, o[0]);
+            lerp_column(make_float2(f00.z, f00.w), make_float2(f01.z, f01.w), make_float2(f10.z, f10.w),
+                        make_float2(f11.z, f11.w), cg, o[1]);
           } else {
-#pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-              // 4 bf16 channels = half of a 16-byte chunk of the 64-channel line
-              const uint32_t g8 = static_cast<uint32_t>(hsel * 4 + gg * 2 + (cq >> 1)) << 4;
-              const uint32_t h8 = static_cast<uint32_t>(cq & 1) << 3;
-              const uint2 u00 = ld_shared_u2(((sp + loff[hs][0]) | (g8 ^ lxs[hs][0])) + h8);
-              const uint2 u01 = ld_shared_u2(((sp + loff[hs][1]) | (g8 ^ lxs[hs][1])) + h8);
-              const uint2 u10 = ld_shared_u2(((sp + loff[hs][2]) | (g8 ^ lxs[hs][2])) + h8);
-              const uint2 u11 = ld_shared_u2(((sp + loff[hs][3]) | (g8 ^ lxs[hs][3])) + h8);
-              lerp_column(bf16lo_hi(u00.x), bf16lo_hi(u01.x), bf16lo_hi(u10.x), bf16lo_hi(u11.x), cg, o[2 * gg]);
-              lerp_column(bf16lo_hi(u00.y), bf16lo_hi(u01.y), bf16lo_hi(u10.y), bf16lo_hi(u11.y), cg, o[2 * gg + 1]);
-            }
+            const uint2 u00 = ld_shared_u2(sp + toff[hs][0]);
+            const uint2 u01 = ld_shared_u2(sp + toff[hs][1]);
+            const uint2 u10 = ld_shared_u2(sp + toff[hs][2]);
+            const uint2 u11 = ld_shared_u2(sp + toff[hs][3]);
+            lerp_column(bf16lo_hi(u00.x), bf16lo_hi(u01.x), bf16lo_hi(u10.x), bf16lo_hi(u11.x), cg, o[0]);
+            lerp_column(bf16lo_hi(u00.y), bf16lo_hi(u01.y), bf16lo_hi(u10.y), bf16lo_hi(u11.y), cg, o[1]);
           }
-          const uint32_t acol = tmem + kColA + st * 64 + hs * 32 + hsel * 16;
+          const uint32_t acol = tmem + kColA + st * 64 + hs * 32 + quarter * 8;
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
             // lanes (jx, jx + 8) of the 16-lane half hf = rows 2 hf, 2 hf + 1
-            const uint32_t r[8] = {o[0][2 * hf], o[1][2 * hf], o[0][2 * hf + 1], o[1][2 * hf + 1],
-                                   o[2][2 * hf], o[3][2 * hf], o[2][2 * hf + 1], o[3][2 * hf + 1]};
-            tmem_st_16x256b_x2(acol + (static_cast<uint32_t>(32 * q + 16 * hf) << 16), r);
+            const uint32_t r[4] = {o[0][2 * hf], o[1][2 * hf], o[0][2 * hf + 1], o[1][2 * hf + 1]};
+            tmem_st_16x256b_x1(acol + (static_cast<uint32_t>(32 * q + 16 * hf) << 16), r);
           }
         }
         if (lane == 0 && warp == kWarpProd0) GKD_TR(7, it);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0 && !(skip_first && it == 0)) mbar_arrive(&ctl->afull[st]);
+        if (lane == 0) {
+          mbar_arrive(&ctl->sempty[ss]);                 // slab consumed (loads completed above)
+          if (!(skip_first && it == 0)) mbar_arrive(&ctl->afull[st]);
+        }
         if (lane == 0 && warp == kWarpProd0) GKD_TR(8, it);
         if (++st == kStages) { st = 0; ph ^= 1; }
+        if (++ss == kSlabStages) { ss = 0; sph ^= 1; }
       }
     }
     tmem_wait_st();
@@ -662,6 +717,9 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
 }  // namespace tc
 
 #ifdef GKD_TRACE
+extern "C" __attribute__((visibility("default"))) int gkd_trace_cta(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, tc::g_cta, sizeof(tc::g_cta)));
+}
 extern "C" __attribute__((visibility("default"))) int gkd_trace_read(void* host, int clear) {
   cudaError_t e = cudaMemcpyFromSymbol(host, tc::g_trace, sizeof(tc::g_trace));
   if (e == cudaSuccess && clear) {
