@@ -11,7 +11,7 @@ namespace gkd {
 // Device error word bits (written by kernels, read by gkd_check_device_error).
 enum : unsigned {
   kErrTimeout = 1u << 0,   // a bounded wait ran out
-  kErrBounds = 1u << 1,    // a debug-build bounds check fired
+  kErrBounds = 1u << 1,    // a bounds or placement check fired (the kernel did no work)
 };
 
 // Test hooks for the forced-timeout path (host-set, consumed by the next launch).

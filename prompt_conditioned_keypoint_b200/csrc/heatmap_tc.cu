@@ -177,6 +177,21 @@ __device__ __forceinline__ uint64_t make_bdesc(uint32_t smem_addr) {
          (2ull << 61);
 }
 
+// One 128-channel stage held in ring slot ST: eight K=16 steps (two 64-channel
+// halves x four) into the accumulator at column dcol. The tensor-memory base is
+// 0 (checked after allocation), so every A address and B-descriptor offset is a
+// compile-time constant: the issuing thread only adds them to fixed registers.
+template <int ST>
+__device__ __forceinline__ void issue_stage(uint32_t dcol, uint64_t bdesc0, uint32_t idesc, uint32_t first) {
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const int hs = t >> 2, kk = t & 3;
+    umma_ts_f16(dcol, kColA + ST * 64 + hs * 32 + kk * 8,
+                bdesc0 + static_cast<uint64_t>((ST * kBBytes + hs * kBSubBytes + kk * 32) >> 4), idesc,
+                t == 0 ? first : 1u);
+  }
+}
+
 __device__ __forceinline__ void set_abort(Smem* ctl, unsigned* err, unsigned bits) {
   ctl->abort_flag = 1;
   atomicOr(err, bits);
@@ -367,6 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       if (ctl->unit_end == ~0ull) ctl->unit_end = total_units;
     }
   }
+  if (tid == 0 && ctl->tmem_base != 0) {
+    // the MMA issue path assumes the whole tensor memory starting at column 0
+    // (the only place a 512-column allocation can land); anything else: no work
+    atomicOr(a.err, kErrBounds);
+    ctl->unit_begin = ctl->unit_end = 0;
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
@@ -486,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       trace_sum_n += ci.n;
 #endif
       const int buf = v & 1;
-      const uint32_t dcol = tmem + buf * kMaxN;
+      const uint32_t dcol = buf ? kMaxN : 0u;
       if (v >= 2 && !mbar_wait_bounded(&ctl->accempty[buf], ((v >> 1) & 1) ^ 1, lim, abortp)) {
         if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
         ok = false;
@@ -507,16 +528,13 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
         tc_fence_after();
         if (lane == 0) {
           GKD_TR(2, it);
-          const uint64_t bd = bdesc0 + ((st * kBBytes) >> 4);
-          const uint32_t acol = tmem + kColA + st * 64;
-#pragma unroll
-          for (int hs = 0; hs < 2; ++hs) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              umma_ts_f16(dcol, acol + hs * 32 + kk * 8, bd + ((hs * kBSubBytes + kk * 32) >> 4), idesc,
-                          (ch > 0 || hs > 0 || kk > 0) ? 1u : 0u);
-              if (hs == 0 && kk == 0) GKD_TR(12, it);
-            }
+          const uint32_t first = ch > 0 ? 1u : 0u;
+          if (st == 0) {
+            issue_stage<0>(dcol, bdesc0, idesc, first);
+          } else if (st == 1) {
+            issue_stage<1>(dcol, bdesc0, idesc, first);
+          } else {
+            issue_stage<2>(dcol, bdesc0, idesc, first);
           }
           GKD_TR(15, it);
           umma_commit(&ctl->empty[st]);
