@@ -235,6 +235,21 @@ def run_reference(args, cfg_desc):
     return 0
 
 
+# ----------------------------------------------------------------------------- multi-rank timing
+def max_over_ranks(seconds: float, pg=None, device="cpu") -> float:
+    """The job lasts as long as its slowest rank: max of a per-rank duration."""
+    import torch
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    if pg is not None:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, crops_per_rank: int, steps: int, max_seconds: float) -> float:
+    """Whole-job crops/s: every rank processes its own crops_per_rank crops per step."""
+    return world * crops_per_rank * steps / max_seconds
+
+
 # ----------------------------------------------------------------------------- GPU leg
 def main(argv=None):
     args = parse_args(argv)
@@ -294,11 +309,8 @@ def main(argv=None):
     elapsed_s = t_start.elapsed_time(t_end) / 1e3
     hm_s = sum(a.elapsed_time(b) for a, b in ev_hm) / 1e3 / args.steps
 
-    t = torch.tensor([elapsed_s], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    max_s = float(t.item())
-    value = world * shape.B * args.steps / max_s
+    max_s = max_over_ranks(elapsed_s, pg, dev)
+    value = job_throughput(world, shape.B, args.steps, max_s)
 
     # roofline of the dominant kernel (gkd_heatmap)
     peaks, peak_src = measured_peaks()
@@ -355,10 +367,8 @@ def main(argv=None):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        te = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
-        if pg:
-            pg.all_reduce(te, op=pg.ReduceOp.MAX)
-        line["e2e"] = {"value": world * shape.B * args.e2e_steps / float(te.item()), "unit": UNIT,
+        te = max_over_ranks(e0.elapsed_time(e1) / 1e3, pg, dev)
+        line["e2e"] = {"value": job_throughput(world, shape.B, args.e2e_steps, te), "unit": UNIT,
                        "h2d_bytes_per_step": head.host_input_bytes(host), "d2h_bytes_per_step": head.output_bytes(),
                        "steps": args.e2e_steps}
     gk.gkd_check_device_error(stream)
