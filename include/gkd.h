@@ -6,17 +6,21 @@
  * coordinates.
  *
  * Sources for the operations (titles and sections of the pages that define them):
- *   [CARD]  "Asher-1/GKD_GGUF" model card, section "Model": Architecture bullet
- *           ("parameter-free detection head (bilinear 4x upsample, L2 kernel
- *           norm, 1x1 kernel conv, per-row mask fusion over prompts padded to
- *           80 rows)"), Prompts bullet (Gaussian pooling sigma = 14, "both
- *           (fused per row)"), Output bullet (peak over a 96x96 grid mapped to
- *           the ROI's normalized -1..1 space plus a confidence score).
- *   [SUMM]  "GKDT: General Keypoint Detection Transformer" summary page,
- *           pipeline paragraph (visual prototypes from Gaussian heatmaps on a
- *           support image; kernels convolve over the query image's features).
- *   [NOTES] GKDT reading notes (arxiv-cs-cv-2607-00752), section "Method"
- *           (visual features aggregated into VKP; normalised convolution).
+ *   [CARD]  Asher-1/GKD_GGUF model card, section Model. Architecture bullet:
+ *           the detection head has no parameters; it upsamples the features
+ *           4x bilinearly, L2-normalises the prompt kernels, applies them as
+ *           1x1 convolutions and fuses rows under a mask, with prompts padded
+ *           to 80 rows. Prompts bullet: visual prompts are pooled with a
+ *           Gaussian of sigma 14; text and visual prompts can be combined row
+ *           by row. Output bullet: the peak of each prompt's heatmap on a 96x96
+ *           grid, mapped into the ROI's -1..1 space, with a confidence score.
+ *   [SUMM]  GKDT: General Keypoint Detection Transformer, summary page,
+ *           pipeline paragraph: visual prototypes come from Gaussian weights
+ *           on the support image; the prompt kernels are convolved over the
+ *           query image's features.
+ *   [NOTES] GKDT reading notes (arxiv-cs-cv-2607-00752), section Method:
+ *           support features are aggregated into visual keypoint prototypes;
+ *           the matching is a normalised convolution.
  *
  * Conventions shared by every entry point:
  *   - Tensor arguments are DEVICE pointers owned by the caller. The library
@@ -73,8 +77,8 @@ typedef enum gkd_dtype {
 
 /*
  * Step 1: Gaussian prototype pooling of support features ([CARD] Prompts
- * bullet, "soft-fiber Gaussian pooling, sigma=14"; [SUMM] pipeline paragraph;
- * [NOTES] Method, support features aggregated into visual prototypes).
+ * bullet, Gaussian pooling with sigma 14; [SUMM] pipeline paragraph; [NOTES]
+ * Method, support features aggregated into visual prototypes).
  *
  *   proto[b,k,:] = sum_ij w_ij * support[b,i,j,:] / sum_ij w_ij,
  *   w_ij = exp(-((X_j - x)^2 + (Y_i - y)^2) / (2 sigma^2)),
@@ -97,8 +101,8 @@ GKD_API gkd_status gkd_pool_prototypes(const void* support, gkd_dtype sdt, int B
                                void* stream);
 
 /*
- * Step 2: L2 normalisation of prompt rows ([CARD] Architecture bullet,
- * "L2 kernel norm ... prompts padded to 80 rows"; [NOTES] Method, normalised
+ * Step 2: L2 normalisation of prompt rows ([CARD] Architecture bullet, kernel
+ * rows normalised, prompts padded to 80 rows; [NOTES] Method, normalised
  * convolution).
  *
  *   out[r,:] = rows[r,:] / max(||rows[r,:]||_2, eps)  where mask[r] != 0,
@@ -116,9 +120,9 @@ GKD_API gkd_status gkd_norm_kernels(const float* rows, const uint8_t* mask, int 
  * Steps 3 + 4: bilinear 4x upsample of the query features (align_corners =
  * False, half-pixel source coordinate s = max((d + 0.5)/4 - 0.5, 0), upper
  * neighbour clamped to the last row/column) fused into the 1x1 dynamic-kernel
- * contraction ([CARD] Architecture bullet, "bilinear 4x upsample, ... 1x1
- * kernel conv"; [CARD] Output bullet, 96x96 grid; [SUMM] "kernels convolve over
- * the query image's features"):
+ * contraction ([CARD] Architecture bullet, 4x bilinear upsample and 1x1
+ * prompt kernels; [CARD] Output bullet, 96x96 grid; [SUMM] pipeline paragraph,
+ * prompt kernels convolved over the query features):
  *
  *   heat[b,m,k,Y,X] = sum_c kern[b,m,k,c] * U[b,Y,X,c]   for mask[b,m,k] != 0.
  *
@@ -142,8 +146,9 @@ GKD_API gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, in
 
 /*
  * Step 5: per-row masked fusion across modalities and peak decode ([CARD]
- * Architecture bullet, "per-row mask fusion"; Prompts bullet, "both (fused
- * per row)"; Output bullet, peak -> ROI -1..1 + confidence score).
+ * Architecture bullet, masked fusion per prompt row; Prompts bullet, text and
+ * visual combined row by row; Output bullet, peak mapped to ROI -1..1 plus a
+ * confidence score).
  *
  * For each (b, k): cnt = number of modalities m with mask[b,m,k] != 0;
  *   fused = heat[b,m,k] for the one present modality, or
@@ -171,7 +176,10 @@ GKD_API const char* gkd_last_error(void);
 /*
  * Synchronises `stream`, then reads and clears the calling device's error
  * word. Returns GKD_ERR_TIMEOUT if a kernel's bounded wait ran out since the
- * last check, GKD_ERR_CUDA if the stream reports a CUDA error, else GKD_OK.
+ * last check; GKD_ERR_CUDA if the stream reports a CUDA error or a kernel
+ * recorded another failure (the tensor-core heatmap kernel refuses to run, and
+ * writes nothing, if its tensor-memory allocation does not start at column 0);
+ * else GKD_OK.
  */
 GKD_API gkd_status gkd_check_device_error(void* stream);
 

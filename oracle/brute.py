@@ -4,8 +4,8 @@ TEST INFRASTRUCTURE ONLY (same import rule as gkd_oracle). A second,
 structurally different restatement used to pin the numpy oracle: nested lists,
 Python floats (IEEE double), one output element at a time, and the upsample as
 a direct 4-tap sum per pixel instead of separable interpolation matrices.
-Sources as in gkd_oracle: GKD_GGUF model card "Model" (Architecture, Prompts,
-Output bullets) and the GKDT summary page's pipeline paragraph.
+Sources as in gkd_oracle: GKD_GGUF model card, Model section (Architecture,
+Prompts and Output bullets) and the GKDT summary page, pipeline paragraph.
 """
 from __future__ import annotations
 

@@ -8,25 +8,27 @@ Plain, slow, obviously-correct restatement of the head in float64 numpy. Every
 step is computed from its definition, in the order the sources give, with no
 blocking or fusion (a BLAS matmul serves as the contraction step):
 
-  a1 Gaussian prototype pooling of support features at keypoints
-     ("soft-fiber Gaussian pooling, sigma=14": GKD_GGUF model card, "Model",
-     Prompts bullet; "Gaussian heatmaps on a support image": GKDT summary page,
-     pipeline paragraph; reading notes "Method", visual keypoints -> VKP)
+  a1 Gaussian prototype pooling of support features at keypoints (visual
+     prompts pooled with a Gaussian of sigma 14: GKD_GGUF model card, Model
+     section, Prompts bullet; Gaussian weights on the support image: GKDT
+     summary page, pipeline paragraph; visual keypoint prototypes: GKDT reading
+     notes, Method section)
   a2 L2 normalisation of prompt rows, K padded to 80 with a validity mask
-     ("L2 kernel norm ... prompts padded to 80 rows": model card, "Model",
-     Architecture bullet; "normalised convolution": reading notes "Method")
+     (model card, Model section, Architecture bullet; normalised convolution:
+     reading notes, Method section)
   a3 bilinear 4x upsample of the query feature map, align_corners=False
-     ("bilinear 4x upsample": model card Architecture bullet; 96x96 grid:
-     model card Output bullet)
+     (model card, Architecture bullet; the 96x96 grid: model card, Output
+     bullet)
   a4 1x1 dynamic-kernel contraction heat = sum_c kernel[c] * U[c, p]
-     ("1x1 kernel conv": model card Architecture bullet; "kernels convolve over
-     the query image's features": summary page, pipeline paragraph)
+     (prompts applied as 1x1 kernels: model card, Architecture bullet; kernels
+     convolved over the query features: summary page, pipeline paragraph)
   a5 per-row masked fusion across modalities, mean of those present
-     ("per-row mask fusion": Architecture bullet; "or both (fused per row)":
-     Prompts bullet)
+     (masked fusion per prompt row: model card, Architecture bullet; text and
+     visual prompts combined row by row: Prompts bullet)
   a6 argmax decode to ROI coordinates in -1..1 plus the peak score
-     ("per-prompt heatmap peak over a 96x96 grid -> keypoints in the ROI's
-     normalized -1..1 space + confidence score": model card Output bullet)
+     (each prompt's heatmap peak on the 96x96 grid, mapped to the ROI's
+     normalised -1..1 space, with a confidence score: model card, Output
+     bullet)
 
 Readings taken where the pages are silent (each is listed in the design notes):
   * pooling evaluates the Gaussian at patch centres S*(j+0.5) of the support

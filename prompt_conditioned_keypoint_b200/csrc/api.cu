@@ -157,6 +157,8 @@ gkd_status gkd_check_device_error(void* stream) {
   if (e == cudaSuccess) e = cudaMemcpy(ds->err_word, &zero, sizeof zero, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return fail(GKD_ERR_CUDA, "error word read failed: %s", cudaGetErrorString(e));
   if (word & gkd::kErrTimeout) return fail(GKD_ERR_TIMEOUT, "a kernel's bounded wait timed out (word 0x%x)", word);
+  if (word & gkd::kErrBounds)
+    return fail(GKD_ERR_CUDA, "a kernel's placement or bounds check failed; it did no work (word 0x%x)", word);
   if (word) return fail(GKD_ERR_CUDA, "device error word 0x%x", word);
   return ok();
 }

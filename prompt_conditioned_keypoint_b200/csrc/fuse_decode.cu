@@ -1,9 +1,9 @@
-// Steps a5 + a6: per-row masked fusion across prompt modalities ("per-row mask
-// fusion over prompts padded to 80 rows", GKD_GGUF model card, "Model" section,
-// Architecture bullet; "or both (fused per row)", Prompts bullet), then the
-// peak of each fused heatmap mapped to ROI coordinates in -1..1 with its score
-// ("per-prompt heatmap peak over a 96x96 grid -> keypoints in the ROI's
-// normalized -1..1 space + confidence score", Output bullet).
+// Steps a5 + a6: per-row masked fusion across prompt modalities (prompt rows are
+// padded to 80 and fused row by row under a validity mask, GKD_GGUF model card,
+// Model section, Architecture bullet; text and visual prompts may be combined
+// row by row, Prompts bullet), then the peak of each fused heatmap mapped to ROI
+// coordinates in -1..1 with a confidence score (the output is the per-prompt
+// peak on the 96x96 grid in the ROI's normalised space, Output bullet).
 //
 // fused = H_v or H_t when one modality is present, (H_v + H_t) * 0.5 in fp32 when
 // both are; the peak is the first (lowest row-major index) maximal pixel;

@@ -1,7 +1,8 @@
 // Steps a3 + a4 in fp32 (fp32 operands, fp32 accumulation on the FMA pipe):
 // bilinear 4x upsample (align_corners=False) fused into the 1x1 dynamic-kernel
-// contraction ("bilinear 4x upsample ... 1x1 kernel conv", GKD_GGUF model card,
-// "Model" section, Architecture bullet). Used when the kernel rows are fp32;
+// contraction (the head upsamples the features 4x bilinearly and applies the
+// prompts as 1x1 convolution kernels, GKD_GGUF model card, Model section,
+// Architecture bullet). Used when the kernel rows are fp32;
 // the tensor cores' fp32-input mode (tf32) would not meet a 1e-5 relative bound.
 //
 // One CTA per (crop, 4x32-pixel tile, group of up to 32 valid rows): each

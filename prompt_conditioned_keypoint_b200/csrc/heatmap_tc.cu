@@ -1,9 +1,9 @@
 // Steps a3 + a4 on the tensor cores: bilinear 4x upsample (align_corners=False)
 // of the query feature map fused into the operand staging of the 1x1
 // dynamic-kernel contraction heat[b,m,k,p] = sum_c khat[b,m,k,c] * U[b,p,c]
-// ("bilinear 4x upsample ... 1x1 kernel conv", GKD_GGUF model card, "Model"
-// section, Architecture bullet; "kernels convolve over the query image's
-// features", GKDT summary page, pipeline paragraph).
+// (4x bilinear upsample and prompts applied as 1x1 convolution kernels: GKD_GGUF
+// model card, Model section, Architecture bullet; the prompt kernels are
+// convolved over the query features: GKDT summary page, pipeline paragraph).
 //
 // GEMM view per crop: D[pixel, row] = U[pixel, :] . khat[row, :], M = pixels,
 // N = the crop's valid prompt rows, K = channels. Operands are bf16, the sum is

@@ -1,6 +1,7 @@
-// Step a2: L2 normalisation of prompt rows ("L2 kernel norm", GKD_GGUF model card,
-// "Model" section, Architecture bullet; "normalised convolution", reading notes
-// "Method"). One warp per row: 128-bit loads, fp32 sum of squares, warp-shuffle
+// Step a2: L2 normalisation of prompt rows: the head normalises each kernel row
+// to unit L2 norm (GKD_GGUF model card, Model section, Architecture bullet; the
+// convolution with prompts is a normalised one, GKDT reading notes, Method
+// section). One warp per row: 128-bit loads, fp32 sum of squares, warp-shuffle
 // reduction, IEEE sqrt and division, optional round-to-nearest-even bf16 output.
 #include "gkd_internal.h"
 #include "ptx.cuh"

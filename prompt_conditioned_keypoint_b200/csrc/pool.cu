@@ -1,7 +1,8 @@
 // Step a1: Gaussian prototype pooling of support-image patch features at the
-// annotated keypoints ("1-shot visual keypoints (soft-fiber Gaussian pooling,
-// sigma=14)", GKD_GGUF model card, "Model" section, Prompts bullet; "Gaussian
-// heatmaps on a support image", GKDT summary page, pipeline paragraph).
+// annotated keypoints. Visual prompts are one-shot keypoints pooled with a
+// Gaussian of sigma 14 px (GKD_GGUF model card, Model section, Prompts bullet);
+// the prototypes come from Gaussian weights placed on the support image at the
+// keypoints (GKDT summary page, pipeline paragraph).
 //
 // proto[b,k,:] = sum_ij w_ij F[b,i,j,:] / sum_ij w_ij with
 // w_ij = exp(-((X_j - x)^2 + (Y_i - y)^2) / (2 sigma^2)) at patch centres

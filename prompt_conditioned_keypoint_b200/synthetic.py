@@ -22,7 +22,7 @@ subset of crops can be regenerated alone.
 The five workloads follow the GKDT-L model card: a DINOv3 ViT-L query map of
 24x24 patches (384 px input, patch 16) with C=1024 channels, prompts padded to
 80 rows, a 4x bilinear upsample to a 96x96 heatmap grid, and visual prompts
-pooled with a Gaussian of sigma 14 px (model card "Model" section).
+pooled with a Gaussian of sigma 14 px (GKD_GGUF model card, Model section).
 """
 from __future__ import annotations
 
