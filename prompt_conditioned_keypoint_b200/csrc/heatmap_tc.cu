@@ -70,9 +70,8 @@ constexpr size_t kSmemBytes =
 struct Smem {            // control block placed after the stage and epilogue buffers
   uint64_t sfull[kSlabStages];
   uint64_t sempty[kSlabStages];
-  uint64_t full[kStages];      // kernel rows landed
+  uint64_t ready[kStages];     // kernel rows landed (TMA bytes) and A written (one arrival per producer warp)
   uint64_t empty[kStages];     // MMA done with kernel rows and A operand
-  uint64_t afull[kStages];
   uint64_t accfull[2];
   uint64_t accempty[2];
   uint64_t drain;
@@ -299,9 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       mbar_init(&ctl->sempty[s], kNumProdWarps);
     }
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->ready[s], 1 + kNumProdWarps);   // kernel-row TMA arming + producers
       mbar_init(&ctl->empty[s], 1);
-      mbar_init(&ctl->afull[s], kNumProdWarps);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&ctl->accfull[t], 1);
@@ -467,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
         }
         if (lane == 0) {
           uint8_t* bp = bring + st * kBBytes;
-          uint64_t* fb = &ctl->full[st];
+          uint64_t* fb = &ctl->ready[st];
           mbar_arrive_expect_tx(fb, bytes);
           const int c0 = ch * kChunk;
 #pragma unroll
@@ -484,49 +482,49 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     if (lane == 0) {
       for (uint32_t k = 0; k < kStages && k < it; ++k) {
         const uint32_t last = it - 1 - k;
-        if (!mbar_wait_drain(&ctl->full[last % kStages], (last / kStages) & 1, lim)) atomicOr(a.err, kErrTimeout);
+        // the stage's phase also needs the producers: on an aborted run it may not
+        // complete, and this bounded wait then only delays the exit
+        if (!mbar_wait_drain(&ctl->ready[last % kStages], (last / kStages) & 1, lim)) atomicOr(a.err, kErrTimeout);
       }
     }
     __syncwarp();
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA
-    uint32_t it = 0, v = 0, st = 0, ph = 0;
+    // One thread runs the whole role (crop sizes computed serially, once per
+    // crop): its per-stage path is one wait, eight MMAs and one commit.
+    if (lane == 0) {
+      uint32_t it = 0, v = 0, st = 0, ph = 0;
 #ifdef GKD_TRACE
-    unsigned long long trace_sum_n = 0;
+      unsigned long long trace_sum_n = 0;
 #endif
-    const uint64_t bdesc0 = make_bdesc(smem_u32(bring));
-    int cur_b = -1;
-    CropInfo ci{};
-    bool ok = true;
-    for (unsigned long long u = ubeg; u < uend && ok; ++u) {
-      const int b = static_cast<int>(u / nU);
-      if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
-      if (ci.n == 0) continue;
-      const uint32_t idesc = make_idesc(ci.n);
+      const uint64_t bdesc0 = make_bdesc(smem_u32(bring));
+      int cur_b = -1, n = 0;
+      bool ok = true;
+      for (unsigned long long u = ubeg; u < uend && ok; ++u) {
+        const int b = static_cast<int>(u / nU);
+        if (b != cur_b) { n = crop_n_serial(a, b); cur_b = b; }
+        if (n == 0) continue;
+        const uint32_t idesc = make_idesc(n);
 #ifdef GKD_TRACE
-      trace_sum_n += ci.n;
+        trace_sum_n += n;
 #endif
-      const int buf = v & 1;
-      const uint32_t dcol = buf ? kMaxN : 0u;
-      if (v >= 2 && !mbar_wait_bounded(&ctl->accempty[buf], ((v >> 1) & 1) ^ 1, lim, abortp)) {
-        if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
-        ok = false;
-        break;
-      }
-      if (lane == 0) GKD_TR(13, v);
-      tc_fence_after();
-      for (int ch = 0; ch < nchunks; ++ch, ++it) {
-        if (lane == 0) GKD_TR(4, it);
-        const bool okf = mbar_wait_bounded(&ctl->full[st], ph, lim, abortp);
-        if (lane == 0) GKD_TR(5, it);
-        if (!okf || !mbar_wait_bounded(&ctl->afull[st], ph, lim, abortp)) {
-          if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
+        const int buf = v & 1;
+        const uint32_t dcol = buf ? kMaxN : 0u;
+        if (v >= 2 && !mbar_wait_bounded(&ctl->accempty[buf], ((v >> 1) & 1) ^ 1, lim, abortp)) {
+          set_abort(ctl, a.err, kErrTimeout);
           ok = false;
           break;
         }
-        if (lane == 0) GKD_TR(11, it);
+        GKD_TR(13, v);
         tc_fence_after();
-        if (lane == 0) {
+        for (int ch = 0; ch < nchunks; ++ch, ++it) {
+          GKD_TR(4, it);
+          if (!mbar_wait_bounded(&ctl->ready[st], ph, lim, abortp)) {
+            set_abort(ctl, a.err, kErrTimeout);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           GKD_TR(2, it);
           const uint32_t first = ch > 0 ? 1u : 0u;
           if (st == 0) {
@@ -536,33 +534,28 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
           } else {
             issue_stage<2>(dcol, bdesc0, idesc, first);
           }
-          GKD_TR(15, it);
           umma_commit(&ctl->empty[st]);
           GKD_TR(3, it);
+          if (++st == kStages) { st = 0; ph ^= 1; }
         }
-        __syncwarp();
-        if (++st == kStages) { st = 0; ph ^= 1; }
-      }
-      if (!ok) break;
-      if (lane == 0) {
+        if (!ok) break;
         umma_commit(&ctl->accfull[buf]);
         GKD_TR(14, v);
+        ++v;
       }
-      __syncwarp();
-      ++v;
-    }
-    // drain: every MMA issued by this thread has completed before teardown
-    if (lane == 0 && it > 0) {
-      umma_commit(&ctl->drain);
-      if (!mbar_wait_drain(&ctl->drain, 0, lim)) atomicOr(a.err, kErrTimeout);
-    }
+      // drain: every MMA issued by this thread has completed before teardown
+      if (it > 0) {
+        umma_commit(&ctl->drain);
+        if (!mbar_wait_drain(&ctl->drain, 0, lim)) atomicOr(a.err, kErrTimeout);
+      }
 #ifdef GKD_TRACE
-    if (lane == 0 && blockIdx.x < 1024) {
-      g_cta[blockIdx.x][1] = global_timer_ns();
-      g_cta[blockIdx.x][2] = v;
-      g_cta[blockIdx.x][3] = trace_sum_n;
-    }
+      if (blockIdx.x < 1024) {
+        g_cta[blockIdx.x][1] = global_timer_ns();
+        g_cta[blockIdx.x][2] = v;
+        g_cta[blockIdx.x][3] = trace_sum_n;
+      }
 #endif
+    }
     __syncwarp();
   } else if (warp < kWarpProd0) {
     // ---------------------------------------------------------------- epilogue
@@ -713,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&ctl->sempty[ss]);                 // slab consumed (loads completed above)
-          if (!(skip_first && it == 0)) mbar_arrive(&ctl->afull[st]);
+          if (!(skip_first && it == 0)) mbar_arrive(&ctl->ready[st]);
         }
         if (lane == 0 && warp == kWarpProd0) GKD_TR(8, it);
         if (++st == kStages) { st = 0; ph ^= 1; }
