@@ -153,9 +153,15 @@ __device__ __forceinline__ int crop_n_serial(const HeatmapTcArgs& a, int b) {
   return (off + 15) & ~15;
 }
 
-// Relative cost of one unit with n accumulator columns (measured on B200: a unit
-// costs about 6 us plus about 0.01 us per accumulator column).
-__device__ __forceinline__ long long unit_cost(int n) { return n == 0 ? 0 : n + 640; }
+// Relative cost of one unit with n accumulator columns and nchunks 128-channel
+// stages, in eighths of one epilogue column (measured on B200: a stage takes
+// about 0.77 us and the epilogue about 0.047 us per column; a unit takes
+// whichever of its stages or the draining of the previous unit's accumulator is
+// longer, plus about an eighth of its epilogue time that the draining warps
+// take from the others).
+__device__ __forceinline__ long long unit_cost(int n, int nchunks) {
+  return n == 0 ? 0 : 8 * max(16LL * nchunks, static_cast<long long>(n)) + n;
+}
 
 __device__ __forceinline__ void src_taps(int d, int n, int& i0, int& i1, float& lam) {
   const float s = fmaxf((static_cast<float>(d) + 0.5f) * 0.25f - 0.5f, 0.0f);
@@ -336,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   } else {
     // pass 1: total cost
     long long local = 0;
-    for (int b = tid; b < a.B; b += kThreads) local += unit_cost(crop_n_serial(a, b)) * nU;
+    for (int b = tid; b < a.B; b += kThreads) local += unit_cost(crop_n_serial(a, b), nchunks) * nU;
     for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
     if (lane == 0 && local) atomicAdd(reinterpret_cast<unsigned long long*>(&ctl->total_cost),
                                       static_cast<unsigned long long>(local));
@@ -348,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     long long carry = 0;
     for (int base = 0; base < a.B; base += kThreads) {
       const int b = base + tid;
-      const long long c = (b < a.B) ? unit_cost(crop_n_serial(a, b)) : 0;
+      const long long c = (b < a.B) ? unit_cost(crop_n_serial(a, b), nchunks) : 0;
       const long long tot = c * nU;
       long long incl = tot;
       for (int o = 1; o < 32; o <<= 1) {

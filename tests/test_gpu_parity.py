@@ -237,6 +237,27 @@ def run_config(cfg):
     return _RUNS[cfg]
 
 
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_every_valid_row_of_every_crop_is_written(cfg):
+    """Work partition coverage at full size: every valid heatmap row of every crop
+    is written (a NaN prefill survives nowhere in them), and rows with mask 0 are
+    left as they were."""
+    wl, head = run_config(cfg)
+    head.heat.fill_(float("nan"))
+    head.norm()
+    head.heatmap()
+    sync_check()
+    mask = torch.as_tensor(np.asarray(wl.mask, dtype=bool), device=dev())
+    if mask.shape[0] == 1:
+        mask = mask.expand(wl.B, -1, -1)
+    finite = torch.isfinite(head.heat).all(dim=-1).all(dim=-1)      # [B][M][K]
+    untouched = torch.isnan(head.heat).all(dim=-1).all(dim=-1)
+    assert bool(finite[mask].all()), f"{int((~finite[mask]).sum())} valid rows not fully written"
+    assert bool(untouched[~mask].all()), "a masked-out row was written"
+    head.forward()          # leave the cached run in its computed state for the other tests
+    sync_check()
+
+
 def oracle_rows(wl, crops):
     """Raw (pre-normalisation) rows of the selected crops, pooling first where the workload pools."""
     if wl.support is None:
