@@ -9,17 +9,17 @@
 // N = the crop's valid prompt rows, K = channels. Operands are bf16, the sum is
 // fp32 in tensor memory.
 //
-// Persistent kernel, one CTA per SM, 14 warps, one M=128 tile (4 output rows x
+// Persistent kernel, one CTA per SM, 23 warps, one M=128 tile (4 output rows x
 // 32 output columns, which all read the same two source rows) per work unit:
-//   warp 0       TMA: per 64-channel chunk, a 2x10-patch feature slab (128B
-//                swizzled) and one box of kernel rows per modality (the B
-//                operand) into a 6-stage ring;
-//   warp 1       MMA issuer: tcgen05.mma kind::f16, A from tensor memory, B from
-//                shared memory, into one of two accumulator buffers, so the next
-//                unit accumulates while the epilogue drains the last one;
-//   warps 2-5    epilogue: tcgen05.ld of the accumulator, transpose through a
+//   warp 0       TMA: per 128-channel stage, a 2x10-patch feature slab (128B
+//                swizzled) into a 6-deep ring; warp 1: TMA of the stage's
+//                kernel rows (the B operand, one box per modality) into a 3-deep ring;
+//   warp 2       MMA issuer (one thread): tcgen05.mma kind::f16, A from tensor
+//                memory, B from shared memory, into one of two accumulator
+//                buffers, so the next unit accumulates while the epilogue drains;
+//   warps 3-6    epilogue: tcgen05.ld of the accumulator, transpose through a
 //                padded shared tile, coalesced float4 heatmap rows;
-//   warps 6-13   upsample producers: a thread owns one output column of four
+//   warps 7-22   upsample producers: a thread owns one output column of four
 //                pixels (one x-lerp per source row serves all four), lerps in
 //                fp32 (packed f32x2), rounds to bf16 and writes the A operand
 //                straight into tensor memory with tcgen05.st.16x256b.
