@@ -1,0 +1,43 @@
+"""bench.py host logic that needs no GPU: the roofline peaks source and the gate on
+committed ncu traffic (reported only for the kernel source it was measured on)."""
+import json
+
+import bench
+
+
+def test_traffic_reported_only_for_the_measured_source(tmp_path, monkeypatch):
+    path = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
+    assert bench.committed_traffic(2) is None                      # no file
+    entry = {"dram_bytes_per_launch": 123.0, "kernel_source_digest": bench.kernel_source_digest()}
+    path.write_text(json.dumps({"workload2": entry}))
+    assert bench.committed_traffic(2) == 123.0
+    assert bench.committed_traffic(3) is None                      # other workload: not measured
+    entry["kernel_source_digest"] = "0" * 16                        # kernel changed since the capture
+    path.write_text(json.dumps({"workload2": entry}))
+    assert bench.committed_traffic(2) is None
+    path.write_text("{not json")
+    assert bench.committed_traffic(2) is None
+
+
+def test_digest_covers_the_kernel_sources():
+    d = bench.kernel_source_digest()
+    assert len(d) == 16 and int(d, 16) >= 0
+
+
+def test_peaks_fallback_when_file_is_missing(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.measured_peaks()
+    assert src == "fallback"
+    assert peaks["hbm_gbs"] == bench.FALLBACK_HBM_GBS and peaks["bf16_tflops"] == bench.FALLBACK_BF16_TFLOPS
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 1.0, "bf16_tflops": 2.0}))
+    peaks, src = bench.measured_peaks()
+    assert src == "MEASURED_PEAKS.json" and peaks["bf16_tflops"] == 2.0
+
+
+def test_args_and_warmup_rule():
+    args = bench.parse_args(["--impl", "reference", "--steps", "2", "--warmup", "1"])
+    assert args.impl == "reference" and args.steps == 2
+    import pytest
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])                              # the GPU leg needs >= 3 warm-up steps
