@@ -144,6 +144,40 @@ def test_heatmap_bf16_parity(case):
         assert (rel > 1e-5).mean() < 0.1, (rel > 1e-5).mean()
 
 
+@pytest.mark.parametrize("h,w", [(256, 256), (255, 129)], ids=["256x256", "255x129"])
+def test_heatmap_largest_grid(h, w):
+    """The largest query grid the boundary accepts, and a ragged one: heatmaps of
+    up to 1024x1024, compared with the oracle on sampled output rows (both border
+    bands, the middle, and every column including the ragged right edge)."""
+    wl = S.make_case(41, 1, h, w, 64, 8, 1, feat_dtype="f32", valid="all")
+    kern = S.random_bf16_rows(41, (1, 1, 8, 64), 0.125)
+    got = run_heatmap(wl, kern)
+    H = 4 * h
+    rows = [0, 1, 2, 3, 4, 5, H // 2 - 1, H // 2, H - 3, H - 2, H - 1]
+    ref = O.heatmap_crop(feat64(wl)[0], O.bf16_decode(kern)[0], wl.mask[0], 4, "bf16", out_rows=rows)
+    g = got[0][:, :, rows, :].reshape(8, -1)
+    assert np.isfinite(got[0]).all()
+    assert_rows_close(g, ref.reshape(8, -1), BF16_TOL, f"heatmap {h}x{w}")
+
+
+def test_heatmap_largest_batch():
+    """B = 65535, the largest batch the boundary accepts (one-patch crops, random
+    masks, some crops with no valid row): every valid row is written, rows with
+    mask 0 are not, and sampled crops match the oracle."""
+    B = 65535
+    wl = S.make_case(42, B, 1, 1, 8, 3, 2, feat_dtype="f32", valid="random")
+    kern = S.random_bf16_rows(42, (B, 2, 3, 8), 0.35)
+    got = run_heatmap(wl, kern)
+    finite = np.isfinite(got).all(axis=(-1, -2))
+    mask = wl.mask.astype(bool)
+    assert finite[mask].all() and not finite[~mask].any()
+    crops = [0, 1, 777, 32768, B - 2, B - 1]
+    ref = O.heatmaps(feat64(wl, crops), O.bf16_decode(kern[crops]), wl.mask[crops], 4, "bf16")
+    g, _ = valid_heat_rows(got[crops], wl.mask[crops])
+    r, _ = valid_heat_rows(ref, wl.mask[crops])
+    assert_rows_close(g, r, BF16_TOL, "heatmap B=65535")
+
+
 @pytest.mark.parametrize("case", [
     dict(seed=31, B=1, h=24, w=24, C=1024, K=80, M=1, valid="prefix"),
     dict(seed=32, B=2, h=5, w=7, C=200, K=13, M=2, valid="random"),
