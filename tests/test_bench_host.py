@@ -41,3 +41,11 @@ def test_args_and_warmup_rule():
     import pytest
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])                              # the GPU leg needs >= 3 warm-up steps
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    args = bench.parse_args(["--impl", "reference", "--steps", "1", "--warmup", "1"])
+    assert bench.run_reference(args, {"workload": "w", "workload_id": 2}) == 0
+    assert capsys.readouterr().out == ""                           # no work, no line on other ranks
