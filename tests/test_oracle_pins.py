@@ -319,6 +319,21 @@ def test_decode_xy_golden(golden_dir):
         assert xy[0, 0, 0] == want, (W, col)
 
 
+def test_decode_xy_2d_golden(golden_dir):
+    """Row-major index and both coordinates on square, wide, tall and ragged grids."""
+    path = os.path.join(golden_dir, "decode_xy2d.txt")
+    with open(path) as f:
+        lines = [[int(v) for v in l.split()] for l in f if l.strip() and not l.startswith("#")]
+    for H, W, row, col, index, xn, xd, yn, yd in lines:
+        heat = np.zeros((1, 1, 1, H, W), np.float32)
+        heat[0, 0, 0, row, col] = 2.0
+        _, idx, xy, score, valid = O.fuse_decode(heat, np.ones((1, 1, 1), np.uint8))
+        assert idx[0, 0] == index == row * W + col
+        assert xy[0, 0, 0] == f32_from_fraction(Fraction(xn, xd)), (H, W, "x")
+        assert xy[0, 0, 1] == f32_from_fraction(Fraction(yn, yd)), (H, W, "y")
+        assert score[0, 0] == 2.0 and valid[0, 0] == 1
+
+
 def test_decode_matches_torch_argmax_and_brute():
     heat = RNG.standard_normal((2, 2, 3, 8, 12)).astype(np.float32)
     heat[0, 0, 1, 2, 3] = heat[0, 0, 1, 5, 1] = 7.0       # tie inside one modality
