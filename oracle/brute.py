@@ -72,3 +72,27 @@ def argmax_first(values) -> int:
         if values[p] > values[best]:
             best = p
     return best
+
+
+def contract_first_value(F, h: int, w: int, C: int, kern_row, Y: int, X: int, up: int, rnd=None) -> float:
+    """Heatmap value with the contraction on the source grid: the 4-tap bilinear
+    sum of g[i][j] = sum_c kern_row[c] * F[i][j][c]; `rnd` optionally rounds
+    each feature value first."""
+    total = 0.0
+    for (iy, wy) in taps(Y, h, up):
+        for (ix, wx) in taps(X, w, up):
+            g = 0.0
+            for c in range(C):
+                f = F[iy][ix][c]
+                if rnd is not None:
+                    f = rnd(f)
+                g += kern_row[c] * f
+            total += wy * wx * g
+    return total
+
+
+def mean_row(rows):
+    """Elementwise mean of one or two equal-length rows."""
+    if len(rows) == 1:
+        return list(rows[0])
+    return [(a + b) * 0.5 for a, b in zip(rows[0], rows[1])]
