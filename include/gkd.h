@@ -28,7 +28,10 @@
  *     device memory, and never synchronises the stream (except
  *     gkd_check_device_error). Work is enqueued asynchronously on `stream`
  *     (a cudaStream_t; NULL means the legacy default stream) on the device
- *     that owns the first tensor argument.
+ *     that owns the first tensor argument. That device becomes the calling
+ *     thread's current device and stays current after the call returns, so
+ *     that a following gkd_check_device_error() on the same thread reads the
+ *     error word of the device that ran the work.
  *   - Layouts are dense row-major with the last index contiguous, unless a
  *     batch-stride argument says otherwise. Strides are in ELEMENTS.
  *   - Masks are uint8 with 0 (absent) or 1 (present) per entry.
@@ -179,7 +182,11 @@ GKD_API const char* gkd_last_error(void);
  * last check; GKD_ERR_CUDA if the stream reports a CUDA error or a kernel
  * recorded another failure (the tensor-core heatmap kernel refuses to run, and
  * writes nothing, if its tensor-memory allocation does not start at column 0);
- * else GKD_OK.
+ * else GKD_OK. There is one error word per device, shared by every launch of
+ * this library on that device from any stream or thread. So the result covers
+ * all of them, not only `stream`'s. A failure recorded by a kernel that is
+ * still running elsewhere, between this call's read and its clear, is lost.
+ * Call it when no other launch of the library is in flight on the device.
  */
 GKD_API gkd_status gkd_check_device_error(void* stream);
 
