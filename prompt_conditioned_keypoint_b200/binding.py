@@ -71,10 +71,16 @@ def _ptr(x) -> int | None:
     return x.data_ptr()
 
 
-def _stream(s) -> int | None:
+def _stream(s, ref=None) -> int | None:
+    """cudaStream_t handle of `s`. None means torch's current stream on the
+    device of `ref` (the call's first tensor, whose device runs the work), or
+    on the current device when `ref` is not a CUDA tensor."""
     if s is None:
         import torch
-        return torch.cuda.current_stream().cuda_stream
+        dev = getattr(ref, "device", None)
+        if dev is None or getattr(dev, "type", None) != "cuda":
+            dev = None
+        return torch.cuda.current_stream(dev).cuda_stream
     if isinstance(s, int):
         return s
     return s.cuda_stream
@@ -109,22 +115,22 @@ def gkd_pool_prototypes(support, sdt, B, h, w, C, kpts, kmask, K, sigma_px, stri
                         proto_batch_stride, stream=None):
     _check("gkd_pool_prototypes", lib.gkd_pool_prototypes(
         _ptr(support), sdt, B, h, w, C, _ptr(kpts), _ptr(kmask), K, sigma_px, stride_px, _ptr(proto),
-        proto_batch_stride, _stream(stream)))
+        proto_batch_stride, _stream(stream, support)))
 
 
 def gkd_norm_kernels(rows, mask, Bk, M, K, C, eps, out_dt, out, stream=None):
     _check("gkd_norm_kernels", lib.gkd_norm_kernels(
-        _ptr(rows), _ptr(mask), Bk, M, K, C, eps, out_dt, _ptr(out), _stream(stream)))
+        _ptr(rows), _ptr(mask), Bk, M, K, C, eps, out_dt, _ptr(out), _stream(stream, rows)))
 
 
 def gkd_heatmap(feat, fdt, B, h, w, C, up, kern, kdt, kern_batch_stride, mask, mask_batch_stride, M, K, heat,
                 stream=None):
     _check("gkd_heatmap", lib.gkd_heatmap(
         _ptr(feat), fdt, B, h, w, C, up, _ptr(kern), kdt, kern_batch_stride, _ptr(mask), mask_batch_stride,
-        M, K, _ptr(heat), _stream(stream)))
+        M, K, _ptr(heat), _stream(stream, feat)))
 
 
 def gkd_fuse_decode(heat, mask, mask_batch_stride, B, M, K, H, W, fused, xy, score, idx, valid, stream=None):
     _check("gkd_fuse_decode", lib.gkd_fuse_decode(
         _ptr(heat), _ptr(mask), mask_batch_stride, B, M, K, H, W, _ptr(fused), _ptr(xy), _ptr(score),
-        _ptr(idx), _ptr(valid), _stream(stream)))
+        _ptr(idx), _ptr(valid), _stream(stream, heat)))

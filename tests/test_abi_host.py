@@ -107,3 +107,34 @@ def test_misc_entry_points():
     with pytest.raises(gk.GkdError) as e:
         gk._check("x", SHAPE)
     assert e.value.status == SHAPE
+
+
+def test_default_stream_follows_the_first_tensors_device(monkeypatch):
+    import torch
+
+    seen = []
+
+    class FakeStream:
+        def __init__(self, dev):
+            self.cuda_stream = 1000 + (-1 if dev is None else torch.device(dev).index)
+
+    def fake_current_stream(dev=None):
+        seen.append(dev)
+        return FakeStream(dev)
+
+    monkeypatch.setattr(torch.cuda, "current_stream", fake_current_stream)
+
+    class OnDevice:
+        device = torch.device("cuda", 3)
+
+    assert gk._stream(None, OnDevice()) == 1003 and seen[-1] == torch.device("cuda", 3)
+    assert gk._stream(None, torch.zeros(4)) == 999 and seen[-1] is None       # CPU tensor
+    assert gk._stream(None, 12345) == 999 and seen[-1] is None                 # raw pointer
+    assert gk._stream(None) == 999
+    n = len(seen)
+    assert gk._stream(77, OnDevice()) == 77                                    # explicit handle wins
+
+    class S:
+        cuda_stream = 55
+
+    assert gk._stream(S(), OnDevice()) == 55 and len(seen) == n
