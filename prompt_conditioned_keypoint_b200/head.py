@@ -171,7 +171,11 @@ class GkdHead:
         return sum(t.numel() * t.element_size() for t in (self.xy, self.score, self.idx, self.valid))
 
     def run_host(self, host: dict, out: dict | None = None, stream=None) -> dict:
-        """End to end through the public API: host inputs in, decoded keypoints out."""
+        """End to end through the public API: host inputs in, decoded keypoints out.
+
+        Everything is enqueued on `stream` (default: the current stream of this
+        head's device) and the copies are asynchronous. Synchronise that stream
+        before reading the returned host tensors or reusing `host`."""
         st = stream if stream is not None else torch.cuda.current_stream(self.device)
         self.upload(host, st)
         self.forward(st)
