@@ -43,6 +43,7 @@ def test_norm_validation():
     good = (P, P, 2, 2, 80, 1024, ctypes.c_float(1e-12), BF16, P, None)
     assert _status("gkd_norm_kernels", P, P, 2, 3, 80, 1024, 1e-12, BF16, P, None) == SHAPE
     assert _status("gkd_norm_kernels", P, P, 2, 2, 0, 1024, 1e-12, BF16, P, None) == SHAPE
+    assert _status("gkd_norm_kernels", P, P, -1, 2, 80, 1024, 1e-12, BF16, P, None) == SHAPE
     assert _status("gkd_norm_kernels", P, P, 2, 2, 129, 1024, 1e-12, BF16, P, None) == SHAPE
     assert _status("gkd_norm_kernels", P, P, 2, 2, 80, 1020, 1e-12, BF16, P, None) == SHAPE
     assert _status("gkd_norm_kernels", P, P, 2, 2, 80, 1024, 0.0, BF16, P, None) == ARG
@@ -63,7 +64,12 @@ def test_heatmap_validation():
     assert hm(fdt=5) == ARG
     assert hm(kdt=5) == ARG
     assert hm(M=2, K=81) == SHAPE                       # 2 * 88 > 160 accumulator columns
-    assert hm(M=1, K=128, kdt=BF16, kbs=128 * 1024, mbs=128) != SHAPE or True
+    # M * ceil8(K) = 128 fits: the call passes every host check and stops only at the
+    # pointer query (no device here, or a non-device stand-in pointer on a GPU machine)
+    assert hm(M=1, K=128, kbs=128 * 1024, mbs=128) in (gk.GKD_ERR_CUDA, ARG)
+    assert hm(M=1, K=129, kbs=129 * 1024, mbs=129) == SHAPE and hm(M=0) == SHAPE and hm(M=3) == SHAPE
+    assert hm(mbs=-1) == SHAPE
+    assert hm(kdt=F32, kbs=2 * 81 * 1024, K=81) in (gk.GKD_ERR_CUDA, ARG)   # no accumulator-column limit in fp32
     assert hm(C=1028) == SHAPE
     assert hm(h=0) == SHAPE and hm(w=257) == SHAPE
     assert hm(B=-1) == SHAPE and hm(B=70000) == SHAPE
@@ -96,6 +102,9 @@ def test_fuse_decode_validation():
     assert fd(M=3) == SHAPE and fd(K=0) == SHAPE and fd(H=3, W=5) == SHAPE
     assert fd(heat=None) == ARG and fd(idx=None) == ARG
     assert fd(heat=MIS) == ALIGN and fd(fused=MIS) == ALIGN and fd(xy=P + 2) == ALIGN
+    assert fd(B=70000) == SHAPE and fd(mbs=-1) == SHAPE and fd(K=65536) == SHAPE
+    assert fd(H=46341, W=46341) == SHAPE                 # H*W >= 2^31
+    assert fd(valid=None) == ARG and fd(score=P + 1) == ALIGN
     assert fd(B=0, heat=None, mask=None, xy=None, score=None, idx=None, valid=None) == OK
 
 
