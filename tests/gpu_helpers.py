@@ -51,13 +51,22 @@ def valid_heat_rows(heat: np.ndarray, mask: np.ndarray):
 
 
 def check_decode_against_margin(ref_fused: np.ndarray, ref_valid: np.ndarray, gpu_idx: np.ndarray,
-                                gpu_valid: np.ndarray, tol: float):
+                                gpu_valid: np.ndarray, tol: float, ref_heat: np.ndarray | None = None,
+                                mask: np.ndarray | None = None):
     """Integer outputs bit-exact everywhere; the peak index bit-exact wherever the
-    oracle's top-2 margin exceeds tol * max|ref| of that fused row."""
+    oracle's top-2 margin exceeds tol * max|ref| of that fused row.
+
+    On the remaining near-tie rows several indices are correct. Given the
+    oracle heatmaps `ref_heat` [B][M][K][H][W] and `mask` [B or 1][M][K], the
+    GPU's index must then be a near-maximal pixel of the oracle's fused row:
+    f[idx] >= max f - 2 (tol S + 1e-6 S), S = the largest |value| of the row's
+    present modality heatmaps. This follows from heatmap rows within tol * S of
+    the oracle (checked before) and the fp32 mean. Returns (rows checked
+    exactly, near-tie rows checked for validity)."""
     from oracle.gkd_oracle import top2_margin
     np.testing.assert_array_equal(gpu_valid, ref_valid)
     checked = 0
-    skipped = 0
+    near = 0
     for b in range(ref_fused.shape[0]):
         for k in range(ref_fused.shape[1]):
             if not ref_valid[b, k]:
@@ -67,6 +76,13 @@ def check_decode_against_margin(ref_fused: np.ndarray, ref_valid: np.ndarray, gp
             if top2_margin(f) > tol * np.abs(f).max():
                 assert gpu_idx[b, k] == int(np.argmax(f)), (b, k)
                 checked += 1
-            else:
-                skipped += 1
-    return checked, skipped
+                continue
+            near += 1
+            if ref_heat is None:
+                continue
+            mb = mask[0 if mask.shape[0] == 1 else b]
+            S = max(float(np.abs(ref_heat[b, m, k]).max()) for m in range(mb.shape[0]) if mb[m, k])
+            i = int(gpu_idx[b, k])
+            assert 0 <= i < f.size, (b, k, i)
+            assert f[i] >= f.max() - 2.0 * (tol + 1e-6) * S, (b, k, i, float(f.max() - f[i]), S)
+    return checked, near
