@@ -77,3 +77,16 @@ def test_simulated_device_within_tolerance_passes():
         _, gidx, _, _, gvalid = O.fuse_decode(np.nan_to_num(noisy, nan=0.0).astype(np.float32), mask)
         checked, near = check_decode_against_margin(fused, valid, gidx, gvalid, BF16_TOL, heat, mask)
         assert checked + near == int(valid.sum())
+
+
+def test_smoke_decode_check_agrees_with_the_test_rule():
+    import __graft_entry__ as G
+    heat, fused, idx, valid, mask = _case(5)
+    exact, near = G.check_decode(fused, heat, mask, idx, BF16_TOL)
+    checked, near2 = check_decode_against_margin(fused, valid, idx, valid, BF16_TOL, heat, mask)
+    assert (exact, near) == (checked, near2) and exact + near == int(valid.sum())
+    b, k = next((b, k) for b in range(valid.shape[0]) for k in range(valid.shape[1]) if valid[b, k])
+    bad = idx.copy()
+    bad[b, k] = int(np.argmin(fused[b, k]))
+    with pytest.raises(AssertionError):
+        G.check_decode(fused, heat, mask, bad, BF16_TOL)
