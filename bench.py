@@ -103,6 +103,7 @@ class ClockSampler:
     def __init__(self, index: int, period_s: float = 0.01):
         self.index, self.period = index, period_s
         self.samples = []
+        self.errors = 0
         self._stop = threading.Event()
         self._thread = None
         self.ok = False
@@ -129,8 +130,8 @@ class ClockSampler:
                 sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
                 util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
                 self.samples.append((sm, self._reasons(), util))
-            except Exception:
-                pass
+            except Exception:   # a failed NVML read: counted and reported, never guessed
+                self.errors += 1
             time.sleep(self.period)
 
     def start(self):
@@ -152,7 +153,7 @@ class ClockSampler:
             bits |= s[1]
         return {"sm_mhz": statistics.median([s[0] for s in busy]) if busy else None, "sm_max_mhz": self.max_mhz,
                 "reasons": [n for b, n in self.REASONS.items() if bits & b and b != 0x1],
-                "samples": len(busy)}
+                "samples": len(busy), "failed_reads": self.errors}
 
 
 # ----------------------------------------------------------------------------- CPU oracle legs

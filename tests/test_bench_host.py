@@ -49,3 +49,49 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     args = bench.parse_args(["--impl", "reference", "--steps", "1", "--warmup", "1"])
     assert bench.run_reference(args, {"workload": "w", "workload_id": 2}) == 0
     assert capsys.readouterr().out == ""                           # no work, no line on other ranks
+
+
+def test_clock_sampler_summary_with_a_fake_nvml(monkeypatch):
+    """Median SM clock over non-idle samples, union of throttle reasons, and a
+    count of failed reads (a stand-in for NVML; no GPU)."""
+    import bench
+
+    class FakeNV:
+        NVML_CLOCK_SM = 0
+
+        def __init__(self):
+            self.calls = 0
+
+        def nvmlDeviceGetClockInfo(self, h, kind):
+            self.calls += 1
+            if self.calls % 4 == 0:
+                raise RuntimeError("transient")
+            return 1965 if self.calls % 2 else 1900
+
+        def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+            return 0x4 if self.calls % 3 == 0 else 0x0
+
+        def nvmlDeviceGetUtilizationRates(self, h):
+            class U:
+                gpu = 100
+            return U()
+
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)
+    cs.samples, cs.errors, cs.period = [], 0, 0.0
+    cs.ok, cs.nv, cs.h, cs.max_mhz = True, FakeNV(), None, 1965
+    import threading
+    cs._stop = threading.Event()
+    # run the sampling loop for a fixed number of polls
+    polls = {"n": 0}
+
+    def fake_sleep(_):
+        polls["n"] += 1
+        if polls["n"] >= 12:
+            cs._stop.set()
+
+    monkeypatch.setattr(bench.time, "sleep", fake_sleep)
+    cs._run()
+    s = cs.summary()
+    assert s["failed_reads"] == 3 and s["samples"] == 9
+    assert s["sm_max_mhz"] == 1965 and s["sm_mhz"] in (1900, 1965)
+    assert s["reasons"] == ["sw_power_cap"]
