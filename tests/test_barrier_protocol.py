@@ -1,0 +1,259 @@
+"""CPU model of the tensor-core heatmap kernel's mbarrier protocol (no GPU).
+
+The persistent kernel in csrc/heatmap_tc.cu runs five roles per CTA over its
+range of work units (one unit = 128 output pixels of one crop; crops with no
+valid rows are skipped by every role alike):
+
+  feature-slab TMA   waits sempty[s] to reuse slab slot s, arms sfull[s] with
+                     the slab's bytes (one arrival plus transaction bytes);
+  kernel-row TMA     waits empty[s] to reuse stage s, arms ready[s] with the
+                     kernel rows' bytes;
+  MMA (one thread)   per unit waits accempty[buf] before reusing accumulator
+                     buf (from the third unit on); per stage waits ready[s],
+                     issues, and commits to empty[s]; at the unit's end
+                     commits to accfull[buf]; finally commits to drain;
+  epilogue warps     per unit wait accfull[buf], then each arrives once on
+                     accempty[buf];
+  producer warps     per stage wait sfull[slab slot] and (from the fourth
+                     stage on) empty[s], then each arrives once on
+                     sempty[slab slot] and ready[s].
+
+Barrier counts: sfull 1, sempty = producer warps, ready = 1 + producer warps,
+empty 1, accfull 1, accempty = epilogue warps, drain 1. Ring depths: 6 slab
+slots, 3 stages, 2 accumulators.
+
+Hardware semantics modelled: a phase completes when its pending arrival count
+and its pending transaction bytes both reach zero; a parity wait on P
+succeeds iff the completed-phase count's parity differs from P; transaction
+bytes land asynchronously in any order; a commit arrives once every earlier
+MMA of its thread is done, i.e. commits are delivered in issue order.
+
+Checked under random schedules (each role given a random speed per run): every successful wait sees exactly the phase
+it means (a parity wait cannot tell phase k from k + 2), every arrival lands
+in the phase it is meant for (none counts toward an earlier one), nothing
+over-arrives, the drains end, and no configuration deadlocks.
+"""
+import random
+
+import pytest
+
+SLAB, STAGES = 6, 3
+
+
+class Bar:
+    def __init__(self, name, count):
+        self.name, self.count = name, count
+        self.pending, self.tx, self.completed = count, 0, 0
+
+    def _maybe_complete(self):
+        if self.pending == 0 and self.tx == 0:
+            self.completed += 1
+            self.pending = self.count
+
+    def arrive(self, phase, who):
+        assert self.completed == phase, f"{who}: arrival for phase {phase} on {self.name} in phase {self.completed}"
+        self.pending -= 1
+        assert self.pending >= 0, f"{who}: over-arrival on {self.name}"
+        self._maybe_complete()
+
+    def expect_tx(self, phase, who):
+        assert self.completed == phase, f"{who}: tx armed for phase {phase} on {self.name} in phase {self.completed}"
+        self.tx += 1
+
+    def land_tx(self):
+        assert self.tx > 0
+        self.tx -= 1
+        self._maybe_complete()
+
+
+def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=False, skip_acc_wait=False,
+             check_waits=True):
+    """units: valid-row counts per unit of this CTA (0 = skipped). Returns the
+    number of stages run; raises AssertionError on a protocol violation.
+    `bad_reuse_parity` plants a wrong parity in the producers' reuse wait;
+    `skip_acc_wait` drops the MMA's wait for a drained accumulator. With
+    `check_waits` False only the data-hazard checks at each access run."""
+    rnd = random.Random(seed)
+    bars = {}
+
+    def bar(name, count):
+        bars[name] = Bar(name, count)
+
+    for s in range(SLAB):
+        bar(("sfull", s), 1)
+        bar(("sempty", s), nprod)
+    for s in range(STAGES):
+        bar(("ready", s), 1 + nprod)
+        bar(("empty", s), 1)
+    for t in range(2):
+        bar(("accfull", t), 1)
+        bar(("accempty", t), nepi)
+    bar(("drain",), 1)
+    live = [n for n in units if n > 0]
+    stages = len(live) * nchunks
+    tx_in_flight = []          # barriers with transaction bytes still landing
+    commits = []               # commit targets in issue order: (barrier, phase)
+
+    # each role yields ("wait", bar, parity, expected_completed) | ("arrive", bar, phase)
+    #                 | ("tx", bar, phase) | ("commit", bar, phase)
+    #                 | ("access", bar, phases_needed, what): a read or overwrite of the
+    #                   buffer that `bar` guards, legal once `bar` has completed that many phases
+    def tma_slab():
+        for it in range(stages):
+            s, k = it % SLAB, it // SLAB
+            if it >= SLAB:
+                yield ("wait", ("sempty", s), (k - 1) & 1, k)
+                yield ("access", ("sempty", s), k, "slab slot overwritten before the producers read it")
+            yield ("tx", ("sfull", s), k)
+        for last in range(max(0, stages - SLAB), stages):          # drain
+            yield ("wait", ("sfull", last % SLAB), (last // SLAB) & 1, last // SLAB + 1)
+
+    def tma_rows():
+        for it in range(stages):
+            s, k = it % STAGES, it // STAGES
+            if it >= STAGES:
+                yield ("wait", ("empty", s), (k - 1) & 1, k)
+                yield ("access", ("empty", s), k, "kernel rows overwritten before the MMA read them")
+            yield ("tx", ("ready", s), k)
+        for last in range(max(0, stages - STAGES), stages):        # drain
+            yield ("wait", ("ready", last % STAGES), (last // STAGES) & 1, last // STAGES + 1)
+
+    def mma():
+        it = 0
+        for v in range(len(live)):
+            buf, use = v & 1, v >> 1
+            if v >= 2 and not skip_acc_wait:
+                yield ("wait", ("accempty", buf), (use - 1) & 1, use)
+            if v >= 2:
+                yield ("access", ("accempty", buf), use, "accumulator overwritten before the epilogue drained it")
+            for _ in range(nchunks):
+                s, k = it % STAGES, it // STAGES
+                yield ("wait", ("ready", s), k & 1, k + 1)
+                yield ("access", ("ready", s), k + 1, "stage read before its operands landed")
+                yield ("commit", ("empty", s), k)
+                it += 1
+            yield ("commit", ("accfull", buf), use)
+        if it > 0:
+            yield ("commit", ("drain",), 0)
+            yield ("wait", ("drain",), 0, 1)
+
+    def epilogue():
+        for v in range(len(live)):
+            buf, use = v & 1, v >> 1
+            yield ("wait", ("accfull", buf), use & 1, use + 1)
+            yield ("access", ("accfull", buf), use + 1, "accumulator read before its MMAs completed")
+            yield ("arrive", ("accempty", buf), use)
+
+    def producer():
+        for it in range(stages):
+            ss, ks = it % SLAB, it // SLAB
+            s, k = it % STAGES, it // STAGES
+            yield ("wait", ("sfull", ss), ks & 1, ks + 1)
+            yield ("access", ("sfull", ss), ks + 1, "slab read before its bytes landed")
+            if it >= STAGES:
+                yield ("wait", ("empty", s), (k & 1) if bad_reuse_parity else ((k - 1) & 1), k)
+                yield ("access", ("empty", s), k, "A stage overwritten before the MMA read it")
+            yield ("arrive", ("sempty", ss), ks)
+            yield ("arrive", ("ready", s), k)
+
+    roles = {"tma_slab": tma_slab(), "tma_rows": tma_rows(), "mma": mma()}
+    roles.update({f"epi{i}": epilogue() for i in range(nepi)})
+    roles.update({f"prod{i}": producer() for i in range(nprod)})
+    cur = {name: next(g, None) for name, g in roles.items()}
+    # per-run role speeds, so that skewed interleavings (a slow epilogue, a fast
+    # issuer) are explored too, not only evenly mixed ones
+    speed = {name: rnd.choice([0.02, 1.0, 50.0]) for name in roles}
+
+    while True:
+        runnable = [n for n, op in cur.items()
+                    if op is not None and (op[0] != "wait" or (bars[op[1]].completed & 1) != op[2])]
+        pending = len(tx_in_flight) + (1 if commits else 0)
+        if not runnable and not pending:
+            break
+        if pending and (not runnable or rnd.random() < async_bias):
+            pick = rnd.randrange(pending)
+            if pick < len(tx_in_flight):
+                bars[tx_in_flight.pop(pick)].land_tx()
+            else:
+                target, phase = commits.pop(0)        # commits complete in issue order
+                bars[target].arrive(phase, "commit")
+            continue
+        name = rnd.choices(runnable, weights=[speed[n] for n in runnable])[0]
+        op = cur[name]
+        if op[0] == "wait":
+            got = bars[op[1]].completed
+            if check_waits:
+                assert got == op[3], f"{name}: wait on {op[1]} passed with {got} phases done, meant {op[3]}"
+        elif op[0] == "access":
+            got = bars[op[1]].completed
+            assert got >= op[2], f"{name}: {op[3]} ({op[1]}: {got} phases done, needs {op[2]})"
+        elif op[0] == "arrive":
+            bars[op[1]].arrive(op[2], name)
+        elif op[0] == "tx":
+            b = bars[op[1]]
+            b.expect_tx(op[2], name)
+            b.arrive(op[2], name)                     # arrive.expect_tx: one arrival plus the bytes
+            tx_in_flight.append(op[1])
+        elif op[0] == "commit":
+            commits.append((op[1], op[2]))
+        cur[name] = next(roles[name], None)
+
+    stuck = {n: op for n, op in cur.items() if op is not None}
+    assert not stuck, f"deadlock: {stuck}"
+    return stages
+
+
+@pytest.mark.parametrize("async_bias", [0.05, 0.3, 0.8])
+def test_protocol_random_schedules(async_bias):
+    rnd = random.Random(int(async_bias * 1000))
+    total = 0
+    for trial in range(120):
+        units = [rnd.choice([0, 16, 48, 96, 160]) for _ in range(rnd.randint(0, 9))]
+        total += simulate(units, rnd.randint(1, 9), nprod=rnd.randint(1, 3), nepi=rnd.randint(1, 2),
+                          seed=trial, async_bias=async_bias)
+    assert total > 0
+
+
+def test_protocol_with_the_kernels_warp_counts():
+    # 16 producer warps and 4 epilogue warps, as launched; long unit runs wrap
+    # every ring many times (6 slab slots, 3 stages, 2 accumulators)
+    for trial in range(6):
+        units = [0, 96, 160, 0, 48, 16, 96, 96, 160, 32]
+        simulate(units, 8, nprod=16, nepi=4, seed=trial, async_bias=0.3)
+
+
+def test_model_catches_a_wrong_reuse_parity():
+    """The check has teeth: producers that wait on empty[s] with the parity of
+    the phase they are about to need, instead of the previous use's, pass on a
+    phase that has not completed, and the model reports it."""
+    for trial in range(20):
+        with pytest.raises(AssertionError):
+            simulate([96, 48, 160, 16], 6, nprod=2, nepi=1, seed=trial, async_bias=0.3,
+                     bad_reuse_parity=True)
+
+
+def test_model_catches_a_missing_accumulator_wait():
+    """Without the MMA's wait on accempty it starts a third unit in an
+    accumulator the epilogue may not have drained: the access check reports the
+    overwrite on some schedule even with the phase-accounting checks off."""
+    failures = 0
+    for trial in range(30):
+        try:
+            simulate([96, 96, 96, 96, 96], 2, nprod=1, nepi=1, seed=trial, async_bias=0.3, skip_acc_wait=True,
+                     check_waits=False)
+        except AssertionError as e:
+            assert "accumulator overwritten" in str(e) or "deadlock" in str(e), str(e)
+            failures += 1
+    assert failures > 0
+
+
+def test_access_checks_alone_catch_a_wrong_reuse_parity():
+    failures = 0
+    for trial in range(20):
+        try:
+            simulate([96, 48, 160, 16], 6, nprod=2, nepi=1, seed=trial, async_bias=0.3, bad_reuse_parity=True,
+                     check_waits=False)
+        except AssertionError as e:
+            assert "overwritten" in str(e) or "deadlock" in str(e) or "phase" in str(e), str(e)
+            failures += 1
+    assert failures > 0
