@@ -47,6 +47,11 @@
  *     kernel records it in a device error word and returns early (outputs are
  *     then unspecified); gkd_check_device_error() reports it as
  *     GKD_ERR_TIMEOUT.
+ *   - Host threads: every entry point may be called from several threads at
+ *     once. gkd_last_error() is per thread. The wait limit
+ *     (gkd_set_wait_timeout_ms) and the debug flags (gkd_debug_set_flags) are
+ *     process-wide: the flags are consumed by whichever bf16 gkd_heatmap
+ *     launch comes next, from any thread.
  */
 #ifndef GKD_H_
 #define GKD_H_
