@@ -96,3 +96,32 @@ def mean_row(rows):
     if len(rows) == 1:
         return list(rows[0])
     return [(a + b) * 0.5 for a, b in zip(rows[0], rows[1])]
+
+
+def preprocess_value(img, H: int, W: int, box, canvas: int, X: int, Y: int, ch: int) -> float:
+    """One normalised output value of the image preprocessing (model card, Model
+    section, Input bullet: longer side resized to the canvas, centre pad with
+    (124, 116, 104), ImageNet normalisation), one pixel at a time: img[y][x][c]
+    nested lists of 0..255 values, box (x0, y0, x1, y1)."""
+    x0, y0, x1, y1 = box
+    bw, bh = x1 - x0, y1 - y0
+    longer = bw if bw > bh else bh
+    s = canvas / longer
+    ox = (canvas - s * bw) / 2.0
+    oy = (canvas - s * bh) / 2.0
+    cx, cy = X + 0.5, Y + 0.5
+    mean = (0.485, 0.456, 0.406)[ch]
+    std = (0.229, 0.224, 0.225)[ch]
+    if not (ox <= cx < ox + s * bw and oy <= cy < oy + s * bh):
+        v = (124.0, 116.0, 104.0)[ch]
+    else:
+        sx = x0 + (cx - ox) / s - 0.5
+        sy = y0 + (cy - oy) / s - 0.5
+        fx, fy = math.floor(sx), math.floor(sy)
+        v = 0.0
+        for (iy, wy) in ((fy, 1.0 - (sy - fy)), (fy + 1, sy - fy)):
+            for (ix, wx) in ((fx, 1.0 - (sx - fx)), (fx + 1, sx - fx)):
+                cyi = min(max(iy, 0), H - 1)
+                cxi = min(max(ix, 0), W - 1)
+                v += wy * wx * img[cyi][cxi][ch]
+    return (v / 255.0 - mean) / std
