@@ -86,12 +86,13 @@ def _normal_nhwc(g: np.random.Generator, C: int, h: int, w: int, scale: float = 
 
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Store fp32 values as bf16 (round to nearest even), returned as uint16 bits.
-
-    A storage cast for input preparation only (torch's conversion)."""
-    import torch
-    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
-    return t.view(torch.int16).numpy().view(np.uint16).copy()
+    """Store finite fp32 values as bf16 (round to nearest, ties to even),
+    returned as uint16 bits. A storage cast for input preparation only: the
+    upper 16 bits after adding 0x7FFF plus the lowest kept bit (the usual
+    integer form of round-half-even on the dropped 16 bits)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = ((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
+    return ((u + r) >> np.uint32(16)).astype(np.uint16)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -213,10 +214,10 @@ def _topdown_workload(seed, crops):
         f = _normal_nhwc(_rng(seed, _FEAT, b), C, h, w, scale=0.5).astype(np.float64)
         uv = _rng(seed, _PEAKS, b).uniform(0.5, 23.5, size=(n, 2))
         centres[t] = uv
-        for k in range(n):
-            gx = np.exp(-0.5 * (jj - uv[k, 0]) ** 2)
-            gy = np.exp(-0.5 * (ii - uv[k, 1]) ** 2)
-            f += amp * (gy[:, None, None] * gx[None, :, None]) * d[k][None, None, :]
+        gx = np.exp(-0.5 * (jj[None, :] - uv[:, 0:1]) ** 2)          # [n][w]
+        gy = np.exp(-0.5 * (ii[None, :] - uv[:, 1:2]) ** 2)          # [n][h]
+        bumps = (gy[:, :, None] * gx[:, None, :]).reshape(n, h * w)  # [n][h*w]
+        f += amp * (bumps.T @ d).reshape(h, w, C)
         feat[t] = to_bf16_bits(f.astype(np.float32))
     return Workload("cfg4", len(sel), h, w, C, K, M, 4, feat, "bf16", rows, mask, 1, "bf16",
                     extra={"centres": centres, "amp": amp})

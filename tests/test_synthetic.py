@@ -51,3 +51,13 @@ def test_bf16_storage_cast_roundtrip():
     back = S.bf16_bits_to_f32(bits)
     assert back[0] == 1.0 and back[2] == -2.5
     assert np.all(np.abs(back - x) <= np.abs(x) * 2.0 ** -8)
+
+
+def test_bf16_storage_cast_matches_torch():
+    import torch
+    g = np.random.default_rng(3)
+    x = np.concatenate([g.standard_normal(200_000).astype(np.float32),
+                        (g.standard_normal(20_000) * 1e-38).astype(np.float32),
+                        np.array([0.0, -0.0, 1.00390625, 1.01171875, -1.00390625, 3.3e38, 1e-45], np.float32)])
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(S.to_bf16_bits(x), want)
