@@ -51,6 +51,9 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true")
+    ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--per-workload-launches", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     return ap.parse_args(argv)
 
@@ -189,7 +192,9 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(wl, budget_s: float):
-    """The oracle as it stands on full crops until the time budget is spent."""
+    """The oracle as it stands on full crops until the time budget is spent,
+    with numpy's BLAS on its default thread pool; plus one crop of workload 1
+    with BLAS held to a single thread."""
     n, t0 = 0, time.perf_counter()
     while True:
         oracle_sample(wl, n % wl.B)
@@ -197,8 +202,24 @@ def cpu_baseline(wl, budget_s: float):
         el = time.perf_counter() - t0
         if el >= budget_s or n >= wl.B:
             break
-    return {"value": n / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} full crop(s) of the same workload, fp64 numpy oracle, {el:.1f} s wall"}
+    out = {"value": n / el, "unit": UNIT, "cores": blas_threads(), "host_cores": os.cpu_count(),
+           "kind": "oracle",
+           "sample": f"{n} full crop(s) of the same workload, fp64 numpy oracle (BLAS matmul for the "
+                     f"contraction, {blas_threads()} BLAS threads), {el:.1f} s wall"}
+    try:
+        from threadpoolctl import threadpool_limits
+
+        from prompt_conditioned_keypoint_b200 import synthetic as S
+        w1 = S.make_config(1)
+        with threadpool_limits(limits=1, user_api="blas"):
+            t1 = time.perf_counter()
+            oracle_sample(w1, 0)
+            t1 = time.perf_counter() - t1
+        out["single_thread_workload1"] = {"value": 1.0 / t1, "unit": UNIT, "cores": 1,
+                                          "sample": "the one crop of workload 1, BLAS on one thread"}
+    except ImportError:
+        out["single_thread_workload1"] = None
+    return out
 
 
 def run_reference(args, cfg_desc):
@@ -249,6 +270,205 @@ def max_over_ranks(seconds: float, pg=None, device="cpu") -> float:
 def job_throughput(world: int, crops_per_rank: int, steps: int, max_seconds: float) -> float:
     """Whole-job crops/s: every rank processes its own crops_per_rank crops per step."""
     return world * crops_per_rank * steps / max_seconds
+
+
+
+# ----------------------------------------------------------------------------- roofline
+def heatmap_algorithmic(shape, mask) -> tuple[float, float]:
+    """Algorithmic FLOPs and HBM bytes of one gkd_heatmap launch, valid rows only:
+    2 R C P FLOPs per crop; bytes = features read once + valid kernel rows
+    (bf16, once per distinct prompt set) + valid heatmap rows written (fp32)."""
+    m = np.asarray(mask).reshape(np.asarray(mask).shape[0], -1).astype(np.float64)
+    rows_per_set = m.sum(axis=1)
+    rows_valid = rows_per_set[0] * shape.B if shape.shared else rows_per_set.sum()
+    kern_rows = rows_per_set.sum()
+    elt = 2 if shape.feat_dtype == "bf16" else 4
+    kelt = 2 if shape.kern_dtype == "bf16" else 4
+    P = shape.H * shape.W
+    flops = 2.0 * rows_valid * shape.C * P
+    hbm = shape.B * shape.h * shape.w * shape.C * elt + kern_rows * shape.C * kelt + rows_valid * P * 4
+    return flops, hbm
+
+
+def heatmap_roofline(shape, mask, launch_s: float, peaks: dict) -> dict:
+    """Roofline of one gkd_heatmap launch of `launch_s` seconds: bf16 operands
+    are bound by the slower of dense bf16 tensor time and HBM time; the fp32
+    path by the FFMA rate (148 SMs x 128 lanes x 2 FLOP x 1.965 GHz)."""
+    flops, hbm = heatmap_algorithmic(shape, mask)
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = hbm / (peaks["hbm_gbs"] * 1e9)
+    achieved = flops / launch_s / 1e12
+    if shape.kern_dtype != "bf16":
+        peak_alu = 148 * 128 * 2 * 1.965e3 / 1e3
+        t_alu = flops / (peak_alu * 1e12)
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s",
+                "frac": achieved / peak_alu, "roofline_us": max(t_alu, t_hbm) * 1e6}
+    elif t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "roofline_us": t_tensor * 1e6}
+    else:
+        ach = hbm / launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "roofline_us": t_hbm * 1e6}
+    roof.update({"algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": hbm,
+                 "launch_us": launch_s * 1e6, "frac_of_kernel_roofline": roof["roofline_us"] / (launch_s * 1e6)})
+    return roof
+
+
+def per_workload_heatmaps(dev, stream, launches: int, peaks: dict, cfgs=(1, 2, 3, 4, 5)) -> dict:
+    """gkd_heatmap alone on each workload at full size: `launches` timed launches
+    (CUDA events around each, on the launching stream) after 3 warm-up ones.
+    Workload 1 fits in L2, so a 256 MB buffer is written between its launches
+    (outside the events); the others move more than L2 per launch."""
+    import torch
+    from prompt_conditioned_keypoint_b200 import binding as gk
+    from prompt_conditioned_keypoint_b200 import synthetic as S
+    from prompt_conditioned_keypoint_b200.head import GkdHead, HeadShape
+    out = {}
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    for cfg in cfgs:
+        wl = S.make_config(cfg)
+        shape = HeadShape.of(wl)
+        head = GkdHead(shape, dev)
+        head.upload(head.host_inputs(wl, pin=False), stream)
+        with torch.cuda.stream(stream):
+            if shape.pooled:
+                head.pool(stream)
+            head.norm(stream)
+            for _ in range(3):
+                head.heatmap(stream)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+        small = cfg == 1
+        for a, b in evs:
+            if small:
+                with torch.cuda.stream(stream):
+                    flush.fill_(1.0)
+            a.record(stream)
+            head.heatmap(stream)
+            b.record(stream)
+        stream.synchronize()
+        gk.gkd_check_device_error(stream)
+        ts = [a.elapsed_time(b) / 1e3 for a, b in evs]
+        roof = heatmap_roofline(shape, wl.mask, sum(ts) / len(ts), peaks)
+        roof.update({"launch_us_median": 1e6 * statistics.median(ts), "launch_us_min": 1e6 * min(ts),
+                     "launches": len(ts), "workload": S.CONFIG_NAMES[cfg],
+                     "crops_per_s_heatmap": shape.B / (sum(ts) / len(ts)),
+                     "l2": "flushed between launches" if small else "inputs larger than L2"})
+        out[f"w{cfg}"] = roof
+        del head
+        torch.cuda.empty_cache()
+    return out
+
+
+def _time_launches(fn, stream, launches: int, flush=None):
+    """Median / mean / min seconds of `fn()` over `launches` timed calls (events on
+    `stream`), after 3 warm-up calls; `flush` (if given) runs before each timed call."""
+    import torch
+    for _ in range(3):
+        fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+    for a, b in evs:
+        if flush is not None:
+            flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    stream.synchronize()
+    ts = [a.elapsed_time(b) / 1e3 for a, b in evs]
+    return statistics.median(ts), sum(ts) / len(ts), min(ts)
+
+
+def variant_timings(dev, stream, launches: int, peaks: dict, cfg: int = 2) -> dict:
+    """The variants beside the graded path, on one workload at full size:
+    - fused_decode: whole head with the decode in the heatmap kernel's epilogue
+      (norm -> heatmap_decode), crops/s;
+    - fuse_rows: fusion by linearity (norm_fuse -> heatmap with M = 1), the
+      heatmap launch against its tensor roofline (flops on the fused rows);
+    - contract_first: contraction on the source grid + upsample, against HBM
+      (features + kernel rows + G written and read + heatmaps written);
+    - pool: the pooling kernel on the pooled workloads (1, 5), against the FFMA
+      rate (its FLOPs exceed its bytes: 2 K h w C per crop over the full grid)."""
+    import torch
+    from prompt_conditioned_keypoint_b200 import binding as gk
+    from prompt_conditioned_keypoint_b200 import synthetic as S
+    from prompt_conditioned_keypoint_b200.head import GkdHead, HeadShape
+    out = {}
+    wl = S.make_config(cfg)
+    shape = HeadShape.of(wl)
+    host = None
+    # fused decode: the whole step
+    head = GkdHead(shape, dev, fused_decode=True)
+    host = head.host_inputs(wl, pin=False)
+    head.upload(host, stream)
+    with torch.cuda.stream(stream):
+        med, mean, mn = _time_launches(lambda: head.forward(stream), stream, launches)
+    out["fused_decode"] = {"workload": S.CONFIG_NAMES[cfg], "ms_per_step": 1e3 * mean, "ms_per_step_median": 1e3 * med,
+                           "crops_per_s": shape.B / mean,
+                           "kernels": "norm, heatmap in decode mode, key finaliser (+ a scratch memset)"}
+    del head
+    # fusion by linearity: the heatmap launch
+    head = GkdHead(shape, dev, fuse_rows=True)
+    head.upload(host, stream)
+    with torch.cuda.stream(stream):
+        if shape.pooled:
+            head.pool(stream)
+        head.norm(stream)
+        med, mean, mn = _time_launches(lambda: head.heatmap(stream), stream, launches)
+    fmask = np.asarray(wl.mask).any(axis=1, keepdims=True).astype(np.uint8)
+    r = heatmap_roofline(shape, fmask, mean, peaks)
+    r.update({"launch_us_median": 1e6 * med, "launch_us_min": 1e6 * mn,
+              "note": "flops counted on prompt rows with any modality present (one contraction per row)"})
+    out["fuse_rows"] = r
+    del head
+    # contract then upsample
+    head = GkdHead(shape, dev)
+    head.upload(host, stream)
+    s = shape
+    G = torch.empty((s.B, s.M, s.K, s.h * s.w), device=dev)
+    kbs = 0 if s.shared else s.M * s.K * s.C
+    mbs = 0 if s.shared else s.M * s.K
+
+    def cf():
+        gk.gkd_heatmap_contract_first(head.feat, gk.GKD_BF16 if s.feat_dtype == "bf16" else gk.GKD_F32, s.B, s.h,
+                                      s.w, s.C, 4, head.khat, kbs, head.mask, mbs, s.M, s.K, G, head.heat, stream)
+    with torch.cuda.stream(stream):
+        if shape.pooled:
+            head.pool(stream)
+        head.norm(stream)
+        med, mean, mn = _time_launches(cf, stream, launches)
+    flops, hbm = heatmap_algorithmic(shape, wl.mask)
+    m = np.asarray(wl.mask).reshape(np.asarray(wl.mask).shape[0], -1).astype(np.float64).sum(1)
+    rows = m[0] * s.B if s.shared else m.sum()
+    hbm_cf = hbm + 2.0 * rows * s.h * s.w * 4          # G written once and read once
+    ach = hbm_cf / mean / 1e9
+    out["contract_first"] = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": ach / peaks["hbm_gbs"], "launch_us": 1e6 * mean, "launch_us_median": 1e6 * med,
+                             "algorithmic_bytes_per_launch": hbm_cf, "algorithmic_flops_per_launch": flops / 16.0,
+                             "kernels": "contraction on the source grid (tcgen05) + upsample"}
+    del head, G
+    torch.cuda.empty_cache()
+    # pooling (FFMA-bound)
+    peak_alu = 148 * 128 * 2 * 1.965e3 / 1e3
+    for pc in (1, 5):
+        wp = S.make_config(pc)
+        hs = HeadShape.of(wp)
+        head = GkdHead(hs, dev)
+        head.upload(head.host_inputs(wp, pin=False), stream)
+        flush = torch.empty(64 << 20, dtype=torch.float32, device=dev) if pc == 1 else None
+        with torch.cuda.stream(stream):
+            med, mean, mn = _time_launches(lambda: head.pool(stream), stream, launches,
+                                           (lambda: flush.fill_(1.0)) if flush is not None else None)
+        nk = float(np.asarray(wp.kmask).sum())
+        pf = 2.0 * nk * hs.h * hs.w * hs.C
+        pb = hs.B * hs.h * hs.w * hs.C * 4 + hs.B * hs.K * hs.C * 4
+        out[f"pool_w{pc}"] = {"bound": "alu", "achieved": pf / mean / 1e12, "peak": peak_alu, "unit": "TFLOP/s",
+                              "frac": pf / mean / 1e12 / peak_alu, "launch_us": 1e6 * mean,
+                              "launch_us_median": 1e6 * med, "algorithmic_flops_per_launch": pf,
+                              "algorithmic_bytes_per_launch": pb, "hbm_gbs": pb / mean / 1e9}
+        del head
+    torch.cuda.empty_cache()
+    gk.gkd_check_device_error(stream)
+    return out
 
 
 # ----------------------------------------------------------------------------- GPU leg
@@ -308,40 +528,19 @@ def main(argv=None):
     barrier()
     gk.gkd_check_device_error(stream)
     elapsed_s = t_start.elapsed_time(t_end) / 1e3
-    hm_s = sum(a.elapsed_time(b) for a, b in ev_hm) / 1e3 / args.steps
+    hm_list = [a.elapsed_time(b) / 1e3 for a, b in ev_hm]
+    hm_s = sum(hm_list) / args.steps
 
     max_s = max_over_ranks(elapsed_s, pg, dev)
     value = job_throughput(world, shape.B, args.steps, max_s)
 
     # roofline of the dominant kernel (gkd_heatmap)
     peaks, peak_src = measured_peaks()
-    flops = head.algorithmic_heatmap_flops(wl.mask)
-    achieved = flops / hm_s / 1e12
-    elt = 2 if shape.feat_dtype == "bf16" else 4
-    rows_valid = float(wl.mask.reshape(wl.mask.shape[0], -1).sum(1).sum()) * (shape.B if shape.shared else 1)
-    hbm_bytes = shape.B * shape.h * shape.w * shape.C * elt + rows_valid * shape.C * 2 / (shape.B if shape.shared else 1) \
-        + rows_valid * shape.H * shape.W * 4
-    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
-    t_hbm = hbm_bytes / (peaks["hbm_gbs"] * 1e9)
-    if shape.kern_dtype == "bf16":
-        bound = "tensor" if t_tensor >= t_hbm else "hbm"
-    else:
-        bound = "alu"
-    if bound == "tensor":
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"]}
-    elif bound == "hbm":
-        ach = hbm_bytes / hm_s / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"]}
-    else:
-        peak_alu = 148 * 128 * 2 * 1.965e3 / 1e3   # fp32 FMA lanes x 2 flop x max clock, TFLOP/s
-        roof = {"bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s", "frac": achieved / peak_alu}
-    traffic = committed_traffic(args.config)
-    roof.update({"traffic": traffic, "kernel": "gkd_heatmap", "peak_source": f"{peak_src} (burst figure)",
-                 "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": hbm_bytes,
-                 "launch_us": hm_s * 1e6, "roofline_us": max(t_tensor, t_hbm) * 1e6,
-                 "frac_of_kernel_roofline": max(t_tensor, t_hbm) / hm_s if bound != "alu" else None})
+    roof = heatmap_roofline(shape, wl.mask, hm_s, peaks)
+    flops = roof["algorithmic_flops_per_launch"]
+    roof.update({"traffic": committed_traffic(args.config), "kernel": "gkd_heatmap",
+                 "peak_source": f"{peak_src} (burst figure)",
+                 "launch_us_median": 1e6 * statistics.median(hm_list), "launch_us_min": 1e6 * min(hm_list)})
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
@@ -373,6 +572,11 @@ def main(argv=None):
                        "h2d_bytes_per_step": head.host_input_bytes(host), "d2h_bytes_per_step": head.output_bytes(),
                        "steps": args.e2e_steps}
     gk.gkd_check_device_error(stream)
+
+    if world == 1 and not args.no_per_workload:
+        line["per_workload"] = per_workload_heatmaps(dev, stream, args.per_workload_launches, peaks)
+    if world == 1 and not args.no_variants:
+        line["variants"] = variant_timings(dev, stream, args.per_workload_launches, peaks)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)

@@ -95,3 +95,36 @@ def test_clock_sampler_summary_with_a_fake_nvml(monkeypatch):
     assert s["failed_reads"] == 3 and s["samples"] == 9
     assert s["sm_max_mhz"] == 1965 and s["sm_mhz"] in (1900, 1965)
     assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_heatmap_roofline_arithmetic():
+    """Algorithmic FLOPs and bytes of a heatmap launch count valid rows only
+    (shared prompt sets: the rows once per crop for FLOPs and heatmaps, once in
+    all for the kernel rows), and the bound is the slower of tensor and HBM time."""
+    import numpy as np
+
+    from prompt_conditioned_keypoint_b200.head import HeadShape
+    shape = HeadShape(B=2, h=24, w=24, C=1024, K=80, M=2, feat_dtype="f32", kern_dtype="bf16")
+    mask = np.zeros((2, 2, 80), np.uint8)
+    mask[0, :, :10] = 1          # 20 rows
+    mask[1, 0, :5] = 1           # 5 rows
+    flops, hbm = bench.heatmap_algorithmic(shape, mask)
+    P = 96 * 96
+    assert flops == 2.0 * 25 * 1024 * P
+    assert hbm == 2 * 576 * 1024 * 4 + 25 * 1024 * 2 + 25 * P * 4
+    shared = HeadShape(B=1000, h=24, w=24, C=1024, K=80, M=2, feat_dtype="bf16", kern_dtype="bf16", shared=True)
+    m1 = np.zeros((1, 2, 80), np.uint8)
+    m1[0, :, :17] = 1
+    f2, h2 = bench.heatmap_algorithmic(shared, m1)
+    assert f2 == 2.0 * 34 * 1000 * 1024 * P
+    assert h2 == 1000 * 576 * 1024 * 2 + 34 * 1024 * 2 + 34 * 1000 * P * 4
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 1.0e6}
+    t = flops / 1e15
+    r = bench.heatmap_roofline(shape, mask, 2 * t, peaks)
+    assert r["bound"] == "tensor" and abs(r["frac"] - 0.5) < 1e-12 and abs(r["roofline_us"] - t * 1e6) < 1e-9
+    f32 = HeadShape(B=1, h=24, w=24, C=1024, K=80, M=1, kern_dtype="f32")
+    r = bench.heatmap_roofline(f32, mask[:1, :1], 1e-3, peaks)
+    assert r["bound"] == "alu"
+    slow_hbm = {"bf16_tflops": 1000.0, "hbm_gbs": 1.0}
+    r = bench.heatmap_roofline(shape, mask, 1.0, slow_hbm)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and abs(r["achieved"] - hbm / 1e9) < 1e-9
