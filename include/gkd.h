@@ -100,8 +100,8 @@ typedef enum gkd_dtype {
  *   proto    fp32; crop b's rows start at proto + b * proto_batch_stride and are
  *            [K][C] contiguous (proto_batch_stride >= K * C; pass 2*K*C to
  *            write straight into modality 0 of a [B][2][K][C] row tensor).
- * Limits: 1 <= K <= 128, 1 <= h, w <= 256, B <= 65535,
- *         4 * K * (2 + h + w) <= 200 KiB, sigma_px > 0, stride_px > 0.
+ * Limits: 1 <= K <= 128, 1 <= h, w <= 256, B <= 65535, sigma_px > 0, stride_px > 0.
+ * The sums are fp32; their order is fixed (it does not depend on scheduling).
  */
 GKD_API gkd_status gkd_pool_prototypes(const void* support, gkd_dtype sdt, int B, int h, int w, int C,
                                const float* kpts, const uint8_t* kmask, int K, float sigma_px,
@@ -123,6 +123,28 @@ GKD_API gkd_status gkd_pool_prototypes(const void* support, gkd_dtype sdt, int B
  */
 GKD_API gkd_status gkd_norm_kernels(const float* rows, const uint8_t* mask, int Bk, int M, int K, int C, float eps,
                             gkd_dtype out_dt, void* out, void* stream);
+
+/*
+ * Step 2 with the modality fusion of step 5 moved in front of the contraction
+ * ("fusion by linearity"): the heatmap is linear in the kernel row, so the mean
+ * of a prompt row's two modality heatmaps ([CARD] Architecture bullet, masked
+ * fusion per row; Prompts bullet, text and visual combined row by row) equals
+ * the heatmap of the mean of its two normalised rows, and the contraction then
+ * runs once per prompt row instead of once per (modality, row).
+ *
+ *   khat_m   = rows[b,m,k,:] / max(||rows[b,m,k,:]||_2, eps)   (as gkd_norm_kernels)
+ *   out[b,k] = (khat_0 + khat_1) * 0.5 in fp32 when both modalities are present,
+ *              khat_m when only m is, 0 when none; rounded once to out_dt
+ *   out_mask[b,k] = 1 if any modality is present, else 0.
+ *   rows [Bk][M][K][C] fp32, mask [Bk][M][K], out [Bk][K][C] (fp32 or bf16),
+ *   out_mask [Bk][K] uint8. Pass out and out_mask to gkd_heatmap or
+ *   gkd_heatmap_decode with M = 1 (and to gkd_fuse_decode with M = 1).
+ * The result differs from the graded fused heatmap only by rounding (a
+ * separately checked variant, not the graded path).
+ * Limits: 1 <= M <= 2, 1 <= K <= 128, eps > 0, Bk*M*K < 2^31.
+ */
+GKD_API gkd_status gkd_norm_fuse_kernels(const float* rows, const uint8_t* mask, int Bk, int M, int K, int C,
+                                         float eps, gkd_dtype out_dt, void* out, uint8_t* out_mask, void* stream);
 
 /*
  * Steps 3 + 4: bilinear 4x upsample of the query features (align_corners =
@@ -153,6 +175,59 @@ GKD_API gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, in
                        float* heat, void* stream);
 
 /*
+ * Steps 3 + 4 in the other order ("contract then upsample", a variant beside
+ * the graded path): the 1x1 contraction and the 4x bilinear upsample ([CARD]
+ * Architecture bullet) are both linear, so
+ *
+ *   G[b,m,k,i,j]   = sum_c kern[b,m,k,c] * bf16(feat[b,i,j,c])   on the h x w grid,
+ *   heat[b,m,k]    = Up(G[b,m,k])   (the rule of gkd_heatmap, applied to G),
+ *
+ * equals gkd_heatmap's result in exact arithmetic with 16x fewer multiply-adds.
+ * Rounding points differ: the features are rounded to bf16 (the tensor-core
+ * operand), U is never formed, G is fp32 (tensor-core accumulation) and the
+ * upsample of G is fp32; so this is checked against its own definition, not
+ * bit for bit against gkd_heatmap. Bound by the heatmap writes (HBM).
+ *
+ * Arguments as in gkd_heatmap with bf16 kernel rows (no kdt), plus
+ *   scratch  [B][M][K][h*w] fp32 device memory owned by the caller (G; rows with
+ *            mask 0 are not written), 4-byte aligned.
+ * Two launches on `stream` (the contraction, then the upsample).
+ * Limits: those of gkd_heatmap's bf16 path.
+ */
+GKD_API gkd_status gkd_heatmap_contract_first(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up,
+                                              const void* kern, long long kern_batch_stride, const uint8_t* mask,
+                                              long long mask_batch_stride, int M, int K, float* scratch,
+                                              float* heat, void* stream);
+
+/*
+ * Steps 3 + 4 + 5 in one pass, heatmaps never written: the contraction of
+ * gkd_heatmap, with the per-row masked fusion and peak decode of
+ * gkd_fuse_decode done on the accumulators inside the heatmap kernel's
+ * epilogue ([CARD] Architecture bullet, masked fusion per prompt row; Output
+ * bullet, per-prompt peak mapped to ROI -1..1 with a confidence score).
+ *
+ * Arguments as in gkd_heatmap (no heat) and gkd_fuse_decode (no fused map);
+ * the outputs idx, xy, score and valid equal gkd_fuse_decode's on the
+ * heatmaps gkd_heatmap writes, bit for bit: the same fp32 fusion of the same
+ * accumulator values and the same first-maximum rule.
+ *   scratch  [B][K] uint64 device memory owned by the caller (8-byte aligned),
+ *            used as one peak key per (crop, row) merged across pixel tiles;
+ *            the call clears it first (asynchronously on `stream`) and leaves
+ *            its contents unspecified. Calls that share a scratch buffer must
+ *            not overlap on the GPU.
+ * Three launches on `stream`: the scratch clear, the heatmap kernel in
+ * decode mode, and a small kernel that turns the keys into the outputs.
+ * NaN values never win; a valid row whose every fused value is NaN decodes to
+ * idx 0 with a NaN score (gkd_fuse_decode does the same).
+ * Limits: those of gkd_heatmap.
+ */
+GKD_API gkd_status gkd_heatmap_decode(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up,
+                                      const void* kern, gkd_dtype kdt, long long kern_batch_stride,
+                                      const uint8_t* mask, long long mask_batch_stride, int M, int K,
+                                      unsigned long long* scratch, float* xy, float* score, int32_t* idx,
+                                      uint8_t* valid, void* stream);
+
+/*
  * Step 5: per-row masked fusion across modalities and peak decode ([CARD]
  * Architecture bullet, masked fusion per prompt row; Prompts bullet, text and
  * visual combined row by row; Output bullet, peak mapped to ROI -1..1 plus a
@@ -167,6 +242,8 @@ GKD_API gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, in
  *           (= 2 (X + 0.5)/W - 1, correctly rounded);
  *   valid = 1.
  * Rows with cnt == 0: idx = -1, xy = (0, 0), score = 0, valid = 0, fused row 0.
+ * Inputs are expected finite. NaN values never win; a valid row whose every
+ * fused value is NaN decodes to idx 0, valid 1 and the (NaN) fused value there.
  *
  *   heat   [B][M][K][H][W] fp32 (rows with mask 0 are not read)
  *   mask   crop b's [M][K] at mask + b * mask_batch_stride (0 = shared)
@@ -177,6 +254,50 @@ GKD_API gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, in
 GKD_API gkd_status gkd_fuse_decode(const float* heat, const uint8_t* mask, long long mask_batch_stride, int B, int M,
                            int K, int H, int W, float* fused, float* xy, float* score, int32_t* idx,
                            uint8_t* valid, void* stream);
+
+/*
+ * Image preprocessing in front of the head ([CARD] Model section, Input
+ * bullet: the ROI's longer side resized to 384 pixels, centre-padded to
+ * 384 x 384 with the mean colour (124, 116, 104), ImageNet normalisation), for
+ * B boxes of one image (one crop per detector box, the top-down use).
+ *
+ * For box b = (x0, y0, x1, y1) (image pixels, edge coordinates: pixel p spans
+ * [p, p + 1)), s = canvas / max(x1 - x0, y1 - y0), ox = (canvas - (x1 - x0) s)/2,
+ * oy likewise (not rounded). Canvas pixel (X, Y) is content iff its centre
+ * (X + 0.5, Y + 0.5) lies in [ox, ox + (x1 - x0) s) x [oy, oy + (y1 - y0) s);
+ * content takes the bilinear sample of the image at
+ * (x0 + (X + 0.5 - ox)/s - 0.5, y0 + (Y + 0.5 - oy)/s - 0.5), each axis' two
+ * taps clamped to the image, no antialiasing; other pixels take the pad colour.
+ * Then out = (v / 255 - mean_c) / std_c, mean (0.485, 0.456, 0.406), std
+ * (0.229, 0.224, 0.225). The page names no filter: this bilinear reading and
+ * the unrounded pad offsets (the geometry of gkd_roi_to_image) are readings.
+ * All arithmetic in fp64, rounded once to fp32.
+ *
+ *   img    [H][W][3] uint8 RGB, device memory
+ *   boxes  [B][4] fp32 (x0, y0, x1, y1), device memory; a box with a
+ *          non-positive or non-finite width or height gives an all-pad canvas
+ *   out    [B][3][canvas][canvas] fp32 (channel-major)
+ * Limits: 1 <= H, W <= 32768, B <= 65535, 1 <= canvas <= 4096 (384 for GKDT-L).
+ */
+GKD_API gkd_status gkd_preprocess(const uint8_t* img, int H, int W, const float* boxes, int B, int canvas,
+                                  float* out, void* stream);
+
+/*
+ * ROI -> original-image coordinates of decoded keypoints ([CARD] Output
+ * bullet, keypoints in the ROI's -1..1 space; Input bullet, the resize and
+ * centre pad that this undoes): canvas pixel p = (u + 1) canvas / 2, then
+ * x = x0 + (p_x - ox) / s, y = y0 + (p_y - oy) / s with s, ox, oy as in
+ * gkd_preprocess. fp64 arithmetic, rounded once to fp32.
+ *
+ *   xy     [B][K][2] fp32 (as gkd_fuse_decode writes it), device memory
+ *   boxes  [B][4] fp32 (x0, y0, x1, y1), device memory; a degenerate box gives NaN
+ *   out    [B][K][2] fp32 image pixels (edge coordinates)
+ * Rows of invalid keypoints are mapped like any other (xy = (0, 0) gives the
+ * box centre); the caller keeps the valid flags.
+ * Limits: B <= 65535, 1 <= K <= 65535, 1 <= canvas <= 4096.
+ */
+GKD_API gkd_status gkd_roi_to_image(const float* xy, const float* boxes, int B, int K, int canvas, float* out,
+                                    void* stream);
 
 /* Message for the last non-OK status returned on the calling thread ("" if none). */
 GKD_API const char* gkd_last_error(void);

@@ -42,8 +42,13 @@ _u = ctypes.c_uint
 _SIGS = {
     "gkd_pool_prototypes": [_p, _i, _i, _i, _i, _i, _p, _p, _i, _f, _f, _p, _ll, _p],
     "gkd_norm_kernels": [_p, _p, _i, _i, _i, _i, _f, _i, _p, _p],
+    "gkd_norm_fuse_kernels": [_p, _p, _i, _i, _i, _i, _f, _i, _p, _p, _p],
     "gkd_heatmap": [_p, _i, _i, _i, _i, _i, _i, _p, _i, _ll, _p, _ll, _i, _i, _p, _p],
     "gkd_fuse_decode": [_p, _p, _ll, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p],
+    "gkd_heatmap_decode": [_p, _i, _i, _i, _i, _i, _i, _p, _i, _ll, _p, _ll, _i, _i, _p, _p, _p, _p, _p, _p],
+    "gkd_preprocess": [_p, _i, _i, _p, _i, _i, _p, _p],
+    "gkd_heatmap_contract_first": [_p, _i, _i, _i, _i, _i, _i, _p, _ll, _p, _ll, _i, _i, _p, _p, _p],
+    "gkd_roi_to_image": [_p, _p, _i, _i, _i, _p, _p],
     "gkd_check_device_error": [_p],
     "gkd_set_wait_timeout_ms": [_u],
     "gkd_debug_set_flags": [_u],
@@ -123,6 +128,11 @@ def gkd_norm_kernels(rows, mask, Bk, M, K, C, eps, out_dt, out, stream=None):
         _ptr(rows), _ptr(mask), Bk, M, K, C, eps, out_dt, _ptr(out), _stream(stream, rows)))
 
 
+def gkd_norm_fuse_kernels(rows, mask, Bk, M, K, C, eps, out_dt, out, out_mask, stream=None):
+    _check("gkd_norm_fuse_kernels", lib.gkd_norm_fuse_kernels(
+        _ptr(rows), _ptr(mask), Bk, M, K, C, eps, out_dt, _ptr(out), _ptr(out_mask), _stream(stream, rows)))
+
+
 def gkd_heatmap(feat, fdt, B, h, w, C, up, kern, kdt, kern_batch_stride, mask, mask_batch_stride, M, K, heat,
                 stream=None):
     _check("gkd_heatmap", lib.gkd_heatmap(
@@ -130,7 +140,31 @@ def gkd_heatmap(feat, fdt, B, h, w, C, up, kern, kdt, kern_batch_stride, mask, m
         M, K, _ptr(heat), _stream(stream, feat)))
 
 
+def gkd_heatmap_decode(feat, fdt, B, h, w, C, up, kern, kdt, kern_batch_stride, mask, mask_batch_stride, M, K,
+                       scratch, xy, score, idx, valid, stream=None):
+    _check("gkd_heatmap_decode", lib.gkd_heatmap_decode(
+        _ptr(feat), fdt, B, h, w, C, up, _ptr(kern), kdt, kern_batch_stride, _ptr(mask), mask_batch_stride,
+        M, K, _ptr(scratch), _ptr(xy), _ptr(score), _ptr(idx), _ptr(valid), _stream(stream, feat)))
+
+
 def gkd_fuse_decode(heat, mask, mask_batch_stride, B, M, K, H, W, fused, xy, score, idx, valid, stream=None):
     _check("gkd_fuse_decode", lib.gkd_fuse_decode(
         _ptr(heat), _ptr(mask), mask_batch_stride, B, M, K, H, W, _ptr(fused), _ptr(xy), _ptr(score),
         _ptr(idx), _ptr(valid), _stream(stream, heat)))
+
+
+def gkd_preprocess(img, H, W, boxes, B, canvas, out, stream=None):
+    _check("gkd_preprocess", lib.gkd_preprocess(_ptr(img), H, W, _ptr(boxes), B, canvas, _ptr(out),
+                                                _stream(stream, img)))
+
+
+def gkd_roi_to_image(xy, boxes, B, K, canvas, out, stream=None):
+    _check("gkd_roi_to_image", lib.gkd_roi_to_image(_ptr(xy), _ptr(boxes), B, K, canvas, _ptr(out),
+                                                    _stream(stream, xy)))
+
+
+def gkd_heatmap_contract_first(feat, fdt, B, h, w, C, up, kern, kern_batch_stride, mask, mask_batch_stride, M, K,
+                               scratch, heat, stream=None):
+    _check("gkd_heatmap_contract_first", lib.gkd_heatmap_contract_first(
+        _ptr(feat), fdt, B, h, w, C, up, _ptr(kern), kern_batch_stride, _ptr(mask), mask_batch_stride, M, K,
+        _ptr(scratch), _ptr(heat), _stream(stream, feat)))

@@ -173,7 +173,6 @@ gkd_status gkd_pool_prototypes(const void* support, gkd_dtype sdt, int B, int h,
   if (C < 8 || C % 8) return fail(GKD_ERR_SHAPE, "C=%d must be a positive multiple of 8", C);
   if (K < 1 || K > 128) return fail(GKD_ERR_SHAPE, "K=%d out of range [1, 128]", K);
   if (!(sigma_px > 0.f) || !(stride_px > 0.f)) return fail(GKD_ERR_ARG, "sigma and stride must be positive");
-  if (4ull * K * (2 + h + w) > 200ull * 1024) return fail(GKD_ERR_SHAPE, "K * (h + w) too large for one CTA");
   if (proto_batch_stride < static_cast<long long>(K) * C)
     return fail(GKD_ERR_SHAPE, "proto_batch_stride=%lld < K*C", proto_batch_stride);
   if (B == 0) return ok();
@@ -213,9 +212,36 @@ gkd_status gkd_norm_kernels(const float* rows, const uint8_t* mask, int Bk, int 
                   "norm");
 }
 
-gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up, const void* kern,
-                       gkd_dtype kdt, long long kern_batch_stride, const uint8_t* mask, long long mask_batch_stride,
-                       int M, int K, float* heat, void* stream) {
+gkd_status gkd_norm_fuse_kernels(const float* rows, const uint8_t* mask, int Bk, int M, int K, int C, float eps,
+                                 gkd_dtype out_dt, void* out, uint8_t* out_mask, void* stream) {
+  if (out_dt != GKD_F32 && out_dt != GKD_BF16) return fail(GKD_ERR_ARG, "out_dt: unknown dtype %d", static_cast<int>(out_dt));
+  if (Bk < 0) return fail(GKD_ERR_SHAPE, "Bk=%d must be >= 0", Bk);
+  if (M < 1 || M > 2) return fail(GKD_ERR_SHAPE, "M=%d must be 1 or 2", M);
+  if (K < 1 || K > 128) return fail(GKD_ERR_SHAPE, "K=%d out of range [1, 128]", K);
+  if (C < 8 || C % 8) return fail(GKD_ERR_SHAPE, "C=%d must be a positive multiple of 8", C);
+  if (!(eps > 0.f)) return fail(GKD_ERR_ARG, "eps must be positive");
+  if (static_cast<long long>(Bk) * M * K >= (1ll << 31)) return fail(GKD_ERR_SHAPE, "too many rows");
+  if (Bk == 0) return ok();
+  if (!rows || !mask || !out || !out_mask) return fail(GKD_ERR_ARG, "null tensor pointer");
+  if (!aligned16(rows) || !aligned16(out)) return fail(GKD_ERR_ALIGN, "rows/out must be 16-byte aligned");
+  int dev = 0;
+  GKD_TRY(use_device_of(rows, "rows", &dev));
+  GKD_TRY(check_same_device(mask, "mask", dev));
+  GKD_TRY(check_same_device(out, "out", dev));
+  GKD_TRY(check_same_device(out_mask, "out_mask", dev));
+  return launched(gkd::launch_norm_fuse(rows, mask, Bk, M, K, C, eps, out_dt == GKD_BF16, out, out_mask,
+                                        static_cast<cudaStream_t>(stream)),
+                  "norm_fuse");
+}
+
+}  // extern "C"
+
+namespace {
+
+// Argument checks shared by gkd_heatmap and gkd_heatmap_decode (no CUDA call).
+gkd_status check_heatmap_args(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up, const void* kern,
+                              gkd_dtype kdt, long long kern_batch_stride, const uint8_t* mask,
+                              long long mask_batch_stride, int M, int K) {
   if (fdt != GKD_F32 && fdt != GKD_BF16) return fail(GKD_ERR_ARG, "fdt: unknown dtype %d", static_cast<int>(fdt));
   if (kdt != GKD_F32 && kdt != GKD_BF16) return fail(GKD_ERR_ARG, "kdt: unknown dtype %d", static_cast<int>(kdt));
   if (kdt == GKD_F32 && fdt != GKD_F32) return fail(GKD_ERR_DTYPE, "fp32 kernel rows need fp32 features");
@@ -228,28 +254,20 @@ gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, int w, int
   if (kdt == GKD_BF16 && M * ((K + 7) / 8 * 8) > 160)
     return fail(GKD_ERR_SHAPE, "M*ceil8(K)=%d exceeds the 160 accumulator columns", M * ((K + 7) / 8 * 8));
   if (kern_batch_stride < 0 || mask_batch_stride < 0) return fail(GKD_ERR_SHAPE, "batch strides must be >= 0");
-  if (B == 0) return ok();
-  if (!feat || !kern || !mask || !heat) return fail(GKD_ERR_ARG, "null tensor pointer");
+  if (B == 0) return GKD_OK;
+  if (!feat || !kern || !mask) return fail(GKD_ERR_ARG, "null tensor pointer");
   const int kelt = kdt == GKD_BF16 ? 2 : 4;
-  if (!aligned16(feat) || !aligned16(kern) || !aligned16(heat) || (kern_batch_stride * kelt) % 16)
-    return fail(GKD_ERR_ALIGN, "feat/kern/heat must be 16-byte aligned and the kernel batch stride a 16-byte multiple");
-  int dev = 0;
-  GKD_TRY(use_device_of(feat, "feat", &dev));
-  GKD_TRY(check_same_device(kern, "kern", dev));
-  GKD_TRY(check_same_device(mask, "mask", dev));
-  GKD_TRY(check_same_device(heat, "heat", dev));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (kdt == GKD_F32)
-    return launched(gkd::launch_heatmap_f32(static_cast<const float*>(feat), B, h, w, C,
-                                            static_cast<const float*>(kern), kern_batch_stride, mask,
-                                            mask_batch_stride, M, K, heat, st),
-                    "heatmap (fp32)");
-  DeviceState* ds = nullptr;
-  GKD_TRY(device_state(dev, &ds));
+  if (!aligned16(feat) || !aligned16(kern) || (kern_batch_stride * kelt) % 16)
+    return fail(GKD_ERR_ALIGN, "feat/kern must be 16-byte aligned and the kernel batch stride a 16-byte multiple");
+  return GKD_OK;
+}
+
+// Fills the tensor-core kernel's arguments (device state looked up by the caller).
+gkd::HeatmapTcArgs tc_args(const DeviceState* ds, gkd_dtype fdt, int B, int h, int w, int C, long long kern_batch_stride,
+                           const uint8_t* mask, long long mask_batch_stride, int M, int K) {
   gkd::HeatmapTcArgs a{};
   a.mask = mask;
   a.mask_batch_stride = mask_batch_stride;
-  a.heat = heat;
   a.B = B;
   a.h = h;
   a.w = w;
@@ -261,10 +279,89 @@ gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, int w, int
   a.err = ds->err_word;
   a.wait_limit_ns = static_cast<unsigned long long>(g_wait_timeout_ms.load()) * 1000000ull;
   a.debug_flags = g_debug_flags.exchange(0);
+  return a;
+}
+
+// The three launches of the decode fused into the heatmap kernel: clear the
+// per-(crop, row) keys, heatmap kernel in decode mode, keys -> outputs.
+gkd_status enqueue_heatmap_decode(int dev, const void* feat, gkd_dtype fdt, int B, int h, int w, int C,
+                                  const void* kern, gkd_dtype kdt, long long kern_batch_stride, const uint8_t* mask,
+                                  long long mask_batch_stride, int M, int K, unsigned long long* keys, float* xy,
+                                  float* score, int32_t* idx, uint8_t* valid, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(keys, 0, sizeof(unsigned long long) * static_cast<size_t>(B) * K, st);
+  if (e != cudaSuccess) return fail(GKD_ERR_CUDA, "scratch clear failed: %s", cudaGetErrorString(e));
+  if (kdt == GKD_F32) {
+    e = gkd::launch_heatmap_f32(static_cast<const float*>(feat), B, h, w, C, static_cast<const float*>(kern),
+                                kern_batch_stride, mask, mask_batch_stride, M, K, nullptr, keys, st);
+    if (e != cudaSuccess) return fail(GKD_ERR_CUDA, "heatmap decode (fp32) launch failed: %s", cudaGetErrorString(e));
+  } else {
+    DeviceState* ds = nullptr;
+    GKD_TRY(device_state(dev, &ds));
+    gkd::HeatmapTcArgs a = tc_args(ds, fdt, B, h, w, C, kern_batch_stride, mask, mask_batch_stride, M, K);
+    a.dec_keys = keys;
+    const char* why = "";
+    e = gkd::launch_heatmap_tc(a, feat, kern, kern_batch_stride, ds->num_sms, st, &why);
+    if (e != cudaSuccess && why[0]) return fail(GKD_ERR_CUDA, "heatmap decode (bf16): %s", why);
+    if (e != cudaSuccess) return fail(GKD_ERR_CUDA, "heatmap decode (bf16) launch failed: %s", cudaGetErrorString(e));
+  }
+  return launched(gkd::launch_finalize_keys(keys, mask, mask_batch_stride, B, M, K, 4 * h, 4 * w, xy, score, idx,
+                                            valid, st),
+                  "decode finalize");
+}
+
+}  // namespace
+
+extern "C" {
+
+gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up, const void* kern,
+                       gkd_dtype kdt, long long kern_batch_stride, const uint8_t* mask, long long mask_batch_stride,
+                       int M, int K, float* heat, void* stream) {
+  GKD_TRY(check_heatmap_args(feat, fdt, B, h, w, C, up, kern, kdt, kern_batch_stride, mask, mask_batch_stride, M, K));
+  if (B == 0) return ok();
+  if (!heat) return fail(GKD_ERR_ARG, "null tensor pointer");
+  if (!aligned16(heat)) return fail(GKD_ERR_ALIGN, "heat must be 16-byte aligned");
+  int dev = 0;
+  GKD_TRY(use_device_of(feat, "feat", &dev));
+  GKD_TRY(check_same_device(kern, "kern", dev));
+  GKD_TRY(check_same_device(mask, "mask", dev));
+  GKD_TRY(check_same_device(heat, "heat", dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (kdt == GKD_F32)
+    return launched(gkd::launch_heatmap_f32(static_cast<const float*>(feat), B, h, w, C,
+                                            static_cast<const float*>(kern), kern_batch_stride, mask,
+                                            mask_batch_stride, M, K, heat, nullptr, st),
+                    "heatmap (fp32)");
+  DeviceState* ds = nullptr;
+  GKD_TRY(device_state(dev, &ds));
+  gkd::HeatmapTcArgs a = tc_args(ds, fdt, B, h, w, C, kern_batch_stride, mask, mask_batch_stride, M, K);
+  a.heat = heat;
   const char* why = "";
   cudaError_t e = gkd::launch_heatmap_tc(a, feat, kern, kern_batch_stride, ds->num_sms, st, &why);
   if (e != cudaSuccess && why[0]) return fail(GKD_ERR_CUDA, "heatmap (bf16): %s", why);
   return launched(e, "heatmap (bf16)");
+}
+
+gkd_status gkd_heatmap_decode(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up, const void* kern,
+                              gkd_dtype kdt, long long kern_batch_stride, const uint8_t* mask,
+                              long long mask_batch_stride, int M, int K, unsigned long long* scratch, float* xy,
+                              float* score, int32_t* idx, uint8_t* valid, void* stream) {
+  GKD_TRY(check_heatmap_args(feat, fdt, B, h, w, C, up, kern, kdt, kern_batch_stride, mask, mask_batch_stride, M, K));
+  if (B == 0) return ok();
+  if (!scratch || !xy || !score || !idx || !valid) return fail(GKD_ERR_ARG, "null tensor pointer");
+  if (reinterpret_cast<uintptr_t>(scratch) & 7u) return fail(GKD_ERR_ALIGN, "scratch must be 8-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(xy) | reinterpret_cast<uintptr_t>(score) | reinterpret_cast<uintptr_t>(idx)) & 3u)
+    return fail(GKD_ERR_ALIGN, "xy/score/idx must be 4-byte aligned");
+  int dev = 0;
+  GKD_TRY(use_device_of(feat, "feat", &dev));
+  GKD_TRY(check_same_device(kern, "kern", dev));
+  GKD_TRY(check_same_device(mask, "mask", dev));
+  GKD_TRY(check_same_device(scratch, "scratch", dev));
+  GKD_TRY(check_same_device(xy, "xy", dev));
+  GKD_TRY(check_same_device(score, "score", dev));
+  GKD_TRY(check_same_device(idx, "idx", dev));
+  GKD_TRY(check_same_device(valid, "valid", dev));
+  return enqueue_heatmap_decode(dev, feat, fdt, B, h, w, C, kern, kdt, kern_batch_stride, mask, mask_batch_stride,
+                                M, K, scratch, xy, score, idx, valid, static_cast<cudaStream_t>(stream));
 }
 
 gkd_status gkd_fuse_decode(const float* heat, const uint8_t* mask, long long mask_batch_stride, int B, int M, int K,
@@ -294,6 +391,78 @@ gkd_status gkd_fuse_decode(const float* heat, const uint8_t* mask, long long mas
   return launched(gkd::launch_fuse_decode(heat, mask, mask_batch_stride, B, M, K, H, W, fused, xy, score, idx, valid,
                                           static_cast<cudaStream_t>(stream)),
                   "fuse_decode");
+}
+
+gkd_status gkd_preprocess(const uint8_t* img, int H, int W, const float* boxes, int B, int canvas, float* out,
+                          void* stream) {
+  if (H < 1 || W < 1 || H > 32768 || W > 32768) return fail(GKD_ERR_SHAPE, "H=%d W=%d out of range [1, 32768]", H, W);
+  if (B < 0 || B > 65535) return fail(GKD_ERR_SHAPE, "B=%d out of range [0, 65535]", B);
+  if (canvas < 1 || canvas > 4096) return fail(GKD_ERR_SHAPE, "canvas=%d out of range [1, 4096]", canvas);
+  if (B == 0) return ok();
+  if (!img || !boxes || !out) return fail(GKD_ERR_ARG, "null tensor pointer");
+  if ((reinterpret_cast<uintptr_t>(boxes) | reinterpret_cast<uintptr_t>(out)) & 3u)
+    return fail(GKD_ERR_ALIGN, "boxes/out must be 4-byte aligned");
+  int dev = 0;
+  GKD_TRY(use_device_of(img, "img", &dev));
+  GKD_TRY(check_same_device(boxes, "boxes", dev));
+  GKD_TRY(check_same_device(out, "out", dev));
+  return launched(gkd::launch_preprocess(img, H, W, boxes, B, canvas, out, static_cast<cudaStream_t>(stream)),
+                  "preprocess");
+}
+
+gkd_status gkd_roi_to_image(const float* xy, const float* boxes, int B, int K, int canvas, float* out, void* stream) {
+  if (B < 0 || B > 65535) return fail(GKD_ERR_SHAPE, "B=%d out of range [0, 65535]", B);
+  if (K < 1 || K > 65535) return fail(GKD_ERR_SHAPE, "K=%d out of range [1, 65535]", K);
+  if (canvas < 1 || canvas > 4096) return fail(GKD_ERR_SHAPE, "canvas=%d out of range [1, 4096]", canvas);
+  if (B == 0) return ok();
+  if (!xy || !boxes || !out) return fail(GKD_ERR_ARG, "null tensor pointer");
+  if ((reinterpret_cast<uintptr_t>(xy) | reinterpret_cast<uintptr_t>(boxes) | reinterpret_cast<uintptr_t>(out)) & 3u)
+    return fail(GKD_ERR_ALIGN, "xy/boxes/out must be 4-byte aligned");
+  int dev = 0;
+  GKD_TRY(use_device_of(xy, "xy", &dev));
+  GKD_TRY(check_same_device(boxes, "boxes", dev));
+  GKD_TRY(check_same_device(out, "out", dev));
+  return launched(gkd::launch_roi_to_image(xy, boxes, B, K, canvas, out, static_cast<cudaStream_t>(stream)),
+                  "roi_to_image");
+}
+
+gkd_status gkd_heatmap_contract_first(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up,
+                                     const void* kern, long long kern_batch_stride, const uint8_t* mask,
+                                     long long mask_batch_stride, int M, int K, float* scratch, float* heat,
+                                     void* stream) {
+  GKD_TRY(check_heatmap_args(feat, fdt, B, h, w, C, up, kern, GKD_BF16, kern_batch_stride, mask, mask_batch_stride,
+                             M, K));
+  if (B == 0) return ok();
+  if (!scratch || !heat) return fail(GKD_ERR_ARG, "null tensor pointer");
+  if (!aligned16(heat) || (reinterpret_cast<uintptr_t>(scratch) & 3u))
+    return fail(GKD_ERR_ALIGN, "heat must be 16-byte aligned and scratch 4-byte aligned");
+  int dev = 0;
+  GKD_TRY(use_device_of(feat, "feat", &dev));
+  GKD_TRY(check_same_device(kern, "kern", dev));
+  GKD_TRY(check_same_device(mask, "mask", dev));
+  GKD_TRY(check_same_device(scratch, "scratch", dev));
+  GKD_TRY(check_same_device(heat, "heat", dev));
+  DeviceState* ds = nullptr;
+  GKD_TRY(device_state(dev, &ds));
+  gkd::ContractArgs a{};
+  a.mask = mask;
+  a.mask_batch_stride = mask_batch_stride;
+  a.G = scratch;
+  a.B = B;
+  a.h = h;
+  a.w = w;
+  a.C = C;
+  a.M = M;
+  a.K = K;
+  a.feat_bf16 = fdt == GKD_BF16;
+  a.kern_shared = kern_batch_stride == 0;
+  a.err = ds->err_word;
+  a.wait_limit_ns = static_cast<unsigned long long>(g_wait_timeout_ms.load()) * 1000000ull;
+  const char* why = "";
+  cudaError_t e = gkd::launch_contract_first(a, feat, kern, kern_batch_stride, heat, static_cast<cudaStream_t>(stream),
+                                             &why);
+  if (e != cudaSuccess && why[0]) return fail(GKD_ERR_CUDA, "contract-first heatmap: %s", why);
+  return launched(e, "contract-first heatmap");
 }
 
 }  // extern "C"

@@ -88,6 +88,12 @@ __global__ void __launch_bounds__(kDecThreads) fuse_decode_kernel(
       if (better(v, i, best, bi)) { best = v; bi = i; }
     }
     if (lane == 0) {
+      if (bi == INT_MAX) {   // no pixel compared (every value NaN): report the first pixel
+        bi = 0;
+        const float a0 = hv ? reinterpret_cast<const float*>(rv)[0] : 0.f;
+        const float c0 = ht ? reinterpret_cast<const float*>(rt)[0] : 0.f;
+        best = (hv && ht) ? __fmul_rn(__fadd_rn(a0, c0), 0.5f) : (hv ? a0 : c0);
+      }
       const int col = bi % W, row = bi / W;
       idx[o] = bi;
       valid[o] = 1;
@@ -96,6 +102,55 @@ __global__ void __launch_bounds__(kDecThreads) fuse_decode_kernel(
       xy[2 * o + 1] = __fdiv_rn(static_cast<float>(2 * row + 1 - H), static_cast<float>(H));
     }
   }
+}
+
+// Decode fused into the heatmap kernels: turn the per-(crop, row) peak keys
+// (decode_key.cuh) into the same outputs as fuse_decode_kernel. One thread per
+// (crop, row).
+__global__ void __launch_bounds__(256) finalize_keys_kernel(const unsigned long long* __restrict__ keys,
+                                                            const uint8_t* __restrict__ mask, long long mask_bs,
+                                                            int B, int M, int K, int H, int W,
+                                                            float* __restrict__ xy, float* __restrict__ score,
+                                                            int32_t* __restrict__ idx, uint8_t* __restrict__ valid) {
+  const long long o = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (o >= static_cast<long long>(B) * K) return;
+  const int b = static_cast<int>(o / K), k = static_cast<int>(o % K);
+  const uint8_t* mb = mask + static_cast<long long>(b) * mask_bs;
+  const bool present = mb[k] != 0 || (M == 2 && mb[K + k] != 0);
+  if (!present) {
+    idx[o] = -1;
+    valid[o] = 0;
+    score[o] = 0.f;
+    xy[2 * o] = 0.f;
+    xy[2 * o + 1] = 0.f;
+    return;
+  }
+  const unsigned long long key = keys[o];
+  int p = 0;
+  float v = __uint_as_float(0x7FC00000u);     // no candidate: every value was NaN
+  if (key != 0) {
+    const uint32_t hi = static_cast<uint32_t>(key >> 32), lo = static_cast<uint32_t>(key);
+    p = static_cast<int>(0x7FFFFFFFu - (lo >> 1));
+    uint32_t u = (hi & 0x80000000u) ? (hi & 0x7FFFFFFFu) : ~hi;
+    if (u == 0 && (lo & 1u)) u = 0x80000000u;    // the peak was -0
+    v = __uint_as_float(u);
+  }
+  const int col = p % W, row = p / W;
+  idx[o] = p;
+  valid[o] = 1;
+  score[o] = v;
+  xy[2 * o] = __fdiv_rn(static_cast<float>(2 * col + 1 - W), static_cast<float>(W));
+  xy[2 * o + 1] = __fdiv_rn(static_cast<float>(2 * row + 1 - H), static_cast<float>(H));
+}
+
+cudaError_t launch_finalize_keys(const unsigned long long* keys, const uint8_t* mask, long long mask_batch_stride,
+                                 int B, int M, int K, int H, int W, float* xy, float* score, int32_t* idx,
+                                 uint8_t* valid, cudaStream_t stream) {
+  const long long n = static_cast<long long>(B) * K;
+  if (n == 0) return cudaSuccess;
+  finalize_keys_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+      keys, mask, mask_batch_stride, B, M, K, H, W, xy, score, idx, valid);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_fuse_decode(const float* heat, const uint8_t* mask, long long mask_batch_stride, int B, int M,

@@ -9,6 +9,12 @@
 // thread owns one pixel, forms its upsampled 32-channel slice in registers
 // (4-tap, dyadic weights) and contracts it against the row chunk staged in
 // shared memory.
+//
+// Decode mode (`keys` non-null): a group holds 16 prompt rows with both
+// modality slots side by side, so each thread fuses its pixel's two heatmap
+// values in fp32 and the CTA merges one peak key per row into `keys` with
+// atomicMax (decode_key.cuh); no heatmap is written.
+#include "decode_key.cuh"
 #include "gkd_internal.h"
 
 namespace gkd {
@@ -26,8 +32,10 @@ __device__ __forceinline__ void taps_f32(int d, int n, int& i0, int& i1, float& 
 
 __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
     const float* __restrict__ feat, int h, int w, int C, const float* __restrict__ kern, long long kern_bs,
-    const uint8_t* __restrict__ mask, long long mask_bs, int M, int K, float* __restrict__ heat) {
+    const uint8_t* __restrict__ mask, long long mask_bs, int M, int K, float* __restrict__ heat,
+    unsigned long long* __restrict__ keys) {
   __shared__ int rows[256];
+  __shared__ int krow[128];
   __shared__ int s_nrows;
   __shared__ float4 ks[kF32Rows][kF32Chunk / 4];
 
@@ -36,10 +44,25 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
   const int ncb = (W + 31) / 32;
   const int band = blockIdx.x / ncb, cb = blockIdx.x % ncb;
   const uint8_t* mb = mask + static_cast<long long>(b) * mask_bs;
+  const bool decode = keys != nullptr;
   if (threadIdx.x == 0) {
     int n = 0;
-    for (int r = 0; r < M * K; ++r)
-      if (mb[r]) rows[n++] = r;
+    if (!decode) {
+      for (int r = 0; r < M * K; ++r)
+        if (mb[r]) rows[n++] = r;
+    } else {
+      // slots 2i, 2i+1: modality 0 and 1 of the i-th prompt row with any modality present (-1: absent)
+      int nk = 0;
+      for (int k = 0; k < K; ++k) {
+        const bool p0 = mb[k] != 0, p1 = M == 2 && mb[K + k] != 0;
+        if (!p0 && !p1) continue;
+        krow[nk] = k;
+        rows[2 * nk] = p0 ? k : -1;
+        rows[2 * nk + 1] = p1 ? K + k : -1;
+        ++nk;
+      }
+      n = 2 * nk;
+    }
     s_nrows = n;
   }
   __syncthreads();
@@ -71,7 +94,8 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
       const int r = t / (kF32Chunk / 4), q = t % (kF32Chunk / 4);
       const int c = c0 + 4 * q;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < nr && c < C) v = __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(rows[r0 + r]) * C + c));
+      if (r < nr && c < C && rows[r0 + r] >= 0)
+        v = __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(rows[r0 + r]) * C + c));
       ks[r][q] = v;
     }
     // this pixel's upsampled channels
@@ -110,6 +134,27 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
     __syncthreads();
   }
 
+  if (decode) {
+    // fuse the two modality slots of each prompt row, then one key per row and warp
+    const bool inside = Y < H && X < W;
+    const uint32_t pixel = inside ? static_cast<uint32_t>(Y * W + X) : 0u;
+    const int lane = threadIdx.x & 31;
+    unsigned long long mine = 0;
+#pragma unroll
+    for (int i = 0; i < kF32Rows / 2; ++i) {
+      if (2 * i < nr) {
+        const bool p0 = rows[r0 + 2 * i] >= 0, p1 = rows[r0 + 2 * i + 1] >= 0;
+        const float f = (p0 && p1) ? __fmul_rn(__fadd_rn(acc[2 * i], acc[2 * i + 1]), 0.5f)
+                                   : (p0 ? acc[2 * i] : acc[2 * i + 1]);
+        uint32_t hi, lo;
+        peak_key(f, pixel, inside, hi, lo);
+        const unsigned long long key = warp_max_key(hi, lo);
+        if (lane == i) mine = key;
+      }
+    }
+    if (mine != 0) atomicMax(keys + static_cast<long long>(b) * K + krow[r0 / 2 + lane], mine);
+    return;
+  }
   if (Y < H && X < W) {
     const long long P = static_cast<long long>(H) * W;
     float* hb = heat + static_cast<long long>(b) * M * K * P + static_cast<long long>(Y) * W + X;
@@ -121,12 +166,13 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
 
 cudaError_t launch_heatmap_f32(const float* feat, int B, int h, int w, int C, const float* kern,
                                long long kern_batch_stride, const uint8_t* mask, long long mask_batch_stride, int M,
-                               int K, float* heat, cudaStream_t stream) {
+                               int K, float* heat, unsigned long long* keys, cudaStream_t stream) {
   if (B == 0) return cudaSuccess;
   const int W = 4 * w;
-  dim3 grid(h * ((W + 31) / 32), (M * K + kF32Rows - 1) / kF32Rows, B);
+  const int groups = keys ? (K + kF32Rows / 2 - 1) / (kF32Rows / 2) : (M * K + kF32Rows - 1) / kF32Rows;
+  dim3 grid(h * ((W + 31) / 32), groups, B);
   heatmap_f32_kernel<<<grid, kF32Threads, 0, stream>>>(feat, h, w, C, kern, kern_batch_stride, mask,
-                                                        mask_batch_stride, M, K, heat);
+                                                        mask_batch_stride, M, K, heat, keys);
   return cudaGetLastError();
 }
 

@@ -9,7 +9,7 @@
 // N = the crop's valid prompt rows, K = channels. Operands are bf16, the sum is
 // fp32 in tensor memory.
 //
-// Persistent kernel, one CTA per SM, 23 warps, one M=128 tile (4 output rows x
+// Persistent kernel, one CTA per SM, 19 warps, one M=128 tile (4 output rows x
 // 32 output columns, which all read the same two source rows) per work unit:
 //   warp 0       TMA: per 128-channel stage, a 2x10-patch feature slab (128B
 //                swizzled) into a 6-deep ring; warp 1: TMA of the stage's
@@ -19,13 +19,19 @@
 //                buffers, so the next unit accumulates while the epilogue drains;
 //   warps 3-6    epilogue: tcgen05.ld of the accumulator, transpose through a
 //                padded shared tile, coalesced float4 heatmap rows;
-//   warps 7-22   upsample producers: a thread owns one output column of four
-//                pixels (one x-lerp per source row serves all four), lerps in
-//                fp32 (packed f32x2), rounds to bf16 and writes the A operand
-//                straight into tensor memory with tcgen05.st.16x256b.
+//   warps 7-18   upsample producers in three groups of four warps (one warp per
+//                tensor-memory lane quadrant); group g builds the A operand of
+//                every stage i with i % 3 == g, so each warp has three stage
+//                periods for its own. A thread owns one output column of four
+//                pixels (one x-lerp per source row serves all four) and 32
+//                channels of the stage, lerps in fp32 (packed f32x2), rounds to
+//                bf16 and writes the A operand straight into tensor memory, one
+//                tcgen05.st.16x256b.x4 per 64 channels and half quadrant.
 // Units are split over CTAs by a static cost-balanced partition computed in the
-// prologue. Every wait is bounded; a timeout sets the device error word and all
-// roles drain their in-flight copies and MMAs and exit.
+// prologue. Every wait is bounded, and every role takes the outcome of a wait
+// as one decision for all of its threads; a timeout sets the device error word
+// and all roles drain their in-flight copies and MMAs and exit.
+#include "decode_key.cuh"
 #include "gkd_internal.h"
 #include "ptx.cuh"
 
@@ -55,22 +61,36 @@ constexpr int kPlaneSplit = 3072;                // plane pitch when each plane 
 constexpr int kSlabBytes = 4 * kPlaneSplit;      // fp32: 4 planes; bf16: 2 planes
 constexpr int kBSubBytes = kMaxN * 128;          // kernel rows of one sub-chunk
 constexpr int kBBytes = 2 * kBSubBytes;          // 40 KB per stage, 1 KB aligned
-constexpr int kEpiCols = 16;                     // accumulator columns per epilogue group
+#ifndef GKD_STORE_REPS
+#define GKD_STORE_REPS 2
+#endif
+constexpr int kStoreReps = GKD_STORE_REPS;       // 16x256b repetitions per producer store (2 or 4)
+static_assert(kStoreReps == 2 || kStoreReps == 4, "producer store width");
+constexpr int kEpiCols = 16;
+constexpr int kDecCols = 8;                      // prompt rows per decode-mode block (len is a multiple of 8)                     // accumulator columns per epilogue group
 constexpr int kEpiStride = 40;                   // floats per (column, row) line of the epilogue tile
 constexpr int kEpiBufBytes = kEpiCols * kUnitRows * kEpiStride * 4;   // 10 KB
-constexpr int kNumProdWarps = 16, kNumEpiWarps = 4;
+// Producer groups take the stages in turn. A group that last built stage i - G
+// waits for the MMA to free A slot i % kStages and for slab slot i % kSlabStages
+// to fill; a parity wait is unambiguous only if the group itself saw the
+// previous phase of both barriers, so G must not exceed kStages and must divide
+// kSlabStages.
+constexpr int kProdGroups = 3, kProdGroupWarps = 4;                 // one warp per lane quadrant
+constexpr int kNumProdWarps = kProdGroups * kProdGroupWarps, kNumEpiWarps = 4;
 constexpr int kNumWarps = 3 + kNumEpiWarps + kNumProdWarps, kThreads = kNumWarps * 32;
 constexpr int kWarpTma = 0, kWarpTmaB = 1, kWarpMma = 2, kWarpEpi0 = 3, kWarpProd0 = 3 + kNumEpiWarps;
 constexpr int kEpiBarrier = 1;                   // named barrier of the four epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColA = 2 * kMaxN;            // accumulators at 0 and 160; A stages at 320 + 64 s
+static_assert(kProdGroups <= kStages && kSlabStages % kProdGroups == 0, "producer groups alias ring phases");
 constexpr size_t kSmemBytes =
     1024 + static_cast<size_t>(kSlabStages) * kSlabBytes + static_cast<size_t>(kStages) * kBBytes + 2 * kEpiBufBytes + 512;
 
 struct Smem {            // control block placed after the stage and epilogue buffers
   uint64_t sfull[kSlabStages];
   uint64_t sempty[kSlabStages];
-  uint64_t ready[kStages];     // kernel rows landed (TMA bytes) and A written (one arrival per producer warp)
+  uint64_t bfull[kStages];     // kernel rows landed (TMA bytes)
+  uint64_t ready[kStages];     // A operand written (one arrival per warp of the stage's producer group)
   uint64_t empty[kStages];     // MMA done with kernel rows and A operand
   uint64_t accfull[2];
   uint64_t accempty[2];
@@ -84,7 +104,6 @@ struct Smem {            // control block placed after the stage and epilogue bu
 struct CropInfo {
   int n;                 // accumulator columns (multiple of 16), 0 = nothing to do
   int kmin0, kmin1, len0, len1, off1;
-  uint32_t vbits[5];     // bit c of word c/32: column c maps to a valid (m, k) row
 };
 
 __device__ __forceinline__ const uint8_t* crop_mask(const HeatmapTcArgs& a, int b) {
@@ -93,11 +112,13 @@ __device__ __forceinline__ const uint8_t* crop_mask(const HeatmapTcArgs& a, int 
 
 // Warp-cooperative: valid-row segments of one crop (all lanes get the result).
 // Segment m covers rows [kmin_m, kmin_m + len_m) of modality m (len a multiple of
-// 8) and lands at accumulator columns [off_m, off_m + len_m), off_0 = 0.
-__device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int lane) {
+// 8) and lands at accumulator columns [off_m, off_m + len_m), off_0 = 0. With
+// `aligned` (decode mode) the segments of the modalities present share one row
+// range, so the two heatmaps of a prompt row sit exactly off_1 columns apart.
+__device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int lane, bool aligned) {
   CropInfo ci;
   const uint8_t* mb = crop_mask(a, b);
-  int kmin[2] = {0, 0}, len[2] = {0, 0};
+  int kmin[2] = {0, 0}, len[2] = {0, 0}, last_[2] = {-1, -1};
 #pragma unroll
   for (int m = 0; m < 2; ++m) {
     if (m >= a.M) continue;
@@ -113,8 +134,14 @@ __device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int
     }
     if (last >= 0) {
       kmin[m] = first;
+      last_[m] = last;
       len[m] = (last - first + 1 + 7) & ~7;
     }
+  }
+  if (aligned && last_[0] >= 0 && last_[1] >= 0) {
+    const int k0 = min(kmin[0], kmin[1]), k1 = max(last_[0], last_[1]);
+    kmin[0] = kmin[1] = k0;
+    len[0] = len[1] = (k1 - k0 + 1 + 7) & ~7;
   }
   ci.kmin0 = kmin[0];
   ci.kmin1 = kmin[1];
@@ -123,34 +150,53 @@ __device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int
   ci.off1 = len[0];
   const int used = len[0] + len[1];
   ci.n = (used + 15) & ~15;
-#pragma unroll
-  for (int g = 0; g < 5; ++g) {
-    const int col = g * 32 + lane;
-    bool v = false;
-    if (col < used) {
-      const bool m1 = col >= ci.off1;
-      const int k = (m1 ? ci.kmin1 : ci.kmin0) + (col - (m1 ? ci.off1 : 0));
-      v = k < a.K && mb[(m1 ? a.K : 0) + k] != 0;
-    }
-    ci.vbits[g] = __ballot_sync(0xffffffffu, v);
-  }
   return ci;
 }
 
-// Thread-local (no warp collectives): number of accumulator columns of a crop.
+// Warp-cooperative: bit c of the result says accumulator column n0 + c (c < 16)
+// holds a valid (m, k) row of crop b.
+__device__ __forceinline__ uint32_t column_bits16(const HeatmapTcArgs& a, int b, const CropInfo& ci, int n0,
+                                                  int lane) {
+  const uint8_t* mb = crop_mask(a, b);
+  const int col = n0 + lane;
+  bool v = false;
+  if (lane < 16 && col < ci.len0 + ci.len1) {
+    const bool m1 = col >= ci.off1;
+    const int k = (m1 ? ci.kmin1 : ci.kmin0) + (col - (m1 ? ci.off1 : 0));
+    v = k < a.K && mb[(m1 ? a.K : 0) + k] != 0;
+  }
+  return __ballot_sync(0xffffffffu, v) & 0xFFFFu;
+}
+
+// Warp-cooperative: whether crop b has any valid row (all lanes get the result).
+__device__ __forceinline__ bool crop_has_rows(const HeatmapTcArgs& a, int b, int lane) {
+  const uint8_t* mb = crop_mask(a, b);
+  const int n = a.M * a.K;
+  bool any = false;
+  for (int i = lane; i < n && !any; i += 32) any = mb[i] != 0;
+  return __any_sync(0xffffffffu, any);
+}
+
+// Thread-local (no warp collectives): number of accumulator columns of a crop
+// (the same count crop_info gives).
 __device__ __forceinline__ int crop_n_serial(const HeatmapTcArgs& a, int b) {
   const uint8_t* mb = crop_mask(a, b);
-  int off = 0;
+  int first[2] = {-1, -1}, last[2] = {-1, -1};
   for (int m = 0; m < a.M; ++m) {
-    int first = -1, last = -1;
     for (int k = 0; k < a.K; ++k)
       if (mb[m * a.K + k]) {
-        if (first < 0) first = k;
-        last = k;
+        if (first[m] < 0) first[m] = k;
+        last[m] = k;
       }
-    if (last >= 0) off += (last - first + 1 + 7) & ~7;
   }
-  return (off + 15) & ~15;
+  int used = 0;
+  if (a.dec_keys != nullptr && last[0] >= 0 && last[1] >= 0) {
+    used = 2 * ((max(last[0], last[1]) - min(first[0], first[1]) + 1 + 7) & ~7);
+  } else {
+    for (int m = 0; m < 2; ++m)
+      if (last[m] >= 0) used += (last[m] - first[m] + 1 + 7) & ~7;
+  }
+  return (used + 15) & ~15;
 }
 
 // Relative cost of one unit with n accumulator columns and nchunks 128-channel
@@ -280,8 +326,70 @@ __device__ __forceinline__ void st_shared_f32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+// One stage (128 channels) of one producer thread: its column of four pixels x
+// 32 channels, written to the A stage at tensor-memory address `acol` (lane
+// quadrant base, column of the stage). Channel group r (0..3) of sub-chunk hs
+// holds channels 64 hs + 16 r + 4 cq .. +3, i.e. columns 8 r + 2 cq, +1 of the
+// sub-chunk: repetition r of the 16x256b.x4 store. fp32 slabs hold 32 channels
+// per 128-byte plane line, bf16 slabs 64.
+template <bool BF16>
+__device__ __forceinline__ void produce_stage(uint32_t sp, const uint32_t (&base)[4], uint32_t plane_bytes,
+                                              uint32_t f20, const Column4& cg, uint32_t acol) {
+  // kStoreReps repetitions of the 16x256b pattern per store: 4 groups per store
+  // (one store per sub-chunk and half quadrant) or 2 (half the live registers)
+#pragma unroll
+  for (int hr = 0; hr < 8 / kStoreReps; ++hr) {
+    const int hs = hr / (4 / kStoreReps);
+    uint32_t rows01[4 * kStoreReps], rows23[4 * kStoreReps];
+#pragma unroll
+    for (int r2 = 0; r2 < kStoreReps; ++r2) {
+      const int r = (hr % (4 / kStoreReps)) * kStoreReps + r2;   // channel group within the sub-chunk
+      uint32_t o[2][4];   // o[p][row]: channel pair p of the group, pixel row 0..3
+      if (!BF16) {
+        const int plane = 2 * hs + (r >> 1);
+        const uint32_t flip = ((static_cast<uint32_t>(r & 1) ^ (f20 & static_cast<uint32_t>(r >> 1))) << 6);
+        const uint32_t pb = sp + static_cast<uint32_t>(plane) * plane_bytes;
+        const float4 f00 = ld_shared_f4(pb + (base[0] ^ flip));
+        const float4 f01 = ld_shared_f4(pb + (base[1] ^ flip));
+        const float4 f10 = ld_shared_f4(pb + (base[2] ^ flip));
+        const float4 f11 = ld_shared_f4(pb + (base[3] ^ flip));
+        lerp_column(make_float2(f00.x, f00.y), make_float2(f01.x, f01.y), make_float2(f10.x, f10.y),
+                    make_float2(f11.x, f11.y), cg, o[0]);
+        lerp_column(make_float2(f00.z, f00.w), make_float2(f01.z, f01.w), make_float2(f10.z, f10.w),
+                    make_float2(f11.z, f11.w), cg, o[1]);
+      } else {
+        const uint32_t flip = (static_cast<uint32_t>(2 * r) ^ (f20 * 4u * static_cast<uint32_t>(hs & 1))) << 4;
+        const uint32_t pb = sp + static_cast<uint32_t>(hs) * plane_bytes;
+        const uint2 u00 = ld_shared_u2(pb + (base[0] ^ flip));
+        const uint2 u01 = ld_shared_u2(pb + (base[1] ^ flip));
+        const uint2 u10 = ld_shared_u2(pb + (base[2] ^ flip));
+        const uint2 u11 = ld_shared_u2(pb + (base[3] ^ flip));
+        lerp_column(bf16lo_hi(u00.x), bf16lo_hi(u01.x), bf16lo_hi(u10.x), bf16lo_hi(u11.x), cg, o[0]);
+        lerp_column(bf16lo_hi(u00.y), bf16lo_hi(u01.y), bf16lo_hi(u10.y), bf16lo_hi(u11.y), cg, o[1]);
+      }
+      // lanes (jx, jx + 8) of a 16-lane half are pixel rows (0, 1) or (2, 3)
+      rows01[4 * r2 + 0] = o[0][0];
+      rows01[4 * r2 + 1] = o[1][0];
+      rows01[4 * r2 + 2] = o[0][1];
+      rows01[4 * r2 + 3] = o[1][1];
+      rows23[4 * r2 + 0] = o[0][2];
+      rows23[4 * r2 + 1] = o[1][2];
+      rows23[4 * r2 + 2] = o[0][3];
+      rows23[4 * r2 + 3] = o[1][3];
+    }
+    const uint32_t col = static_cast<uint32_t>(hs * 32 + (hr % (4 / kStoreReps)) * 8 * kStoreReps);
+    if (kStoreReps == 4) {
+      tmem_st_16x256b_x4(acol + col, reinterpret_cast<const uint32_t(&)[16]>(rows01));
+      tmem_st_16x256b_x4(acol + (16u << 16) + col, reinterpret_cast<const uint32_t(&)[16]>(rows23));
+    } else {
+      tmem_st_16x256b_x2(acol + col, reinterpret_cast<const uint32_t(&)[8]>(rows01));
+      tmem_st_16x256b_x2(acol + (16u << 16) + col, reinterpret_cast<const uint32_t(&)[8]>(rows23));
+    }
+  }
+}
+
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_constant__ HeatmapTcArgs a) {
+__global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ HeatmapTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* bring = smem + kSlabStages * kSlabBytes;          // kernel-row stages
@@ -301,10 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   if (tid == 0) {
     for (int s = 0; s < kSlabStages; ++s) {
       mbar_init(&ctl->sfull[s], 1);
-      mbar_init(&ctl->sempty[s], kNumProdWarps);
+      mbar_init(&ctl->sempty[s], kProdGroupWarps);
     }
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ctl->ready[s], 1 + kNumProdWarps);   // kernel-row TMA arming + producers
+      mbar_init(&ctl->bfull[s], 1);                   // kernel-row TMA arming (+ bytes)
+      mbar_init(&ctl->ready[s], kProdGroupWarps);     // the stage's producer group
       mbar_init(&ctl->empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
@@ -395,7 +504,9 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const unsigned long long ubeg = ctl->unit_begin, uend = ctl->unit_end;
+  // B * nU < 2^32 for every size the boundary accepts (65535 crops x 257 x 32 units)
+  const uint32_t ubeg = static_cast<uint32_t>(ctl->unit_begin), uend = static_cast<uint32_t>(ctl->unit_end);
+  const uint32_t nU32 = static_cast<uint32_t>(nU);
 #ifdef GKD_TRACE
   if (tid == 0 && blockIdx.x < 1024) g_cta[blockIdx.x][0] = global_timer_ns();
 #endif
@@ -407,17 +518,18 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     // ---------------------------------------------------------------- TMA: feature slabs
     uint32_t it = 0, st = 0, ph = 0;
     int cur_b = -1;
-    CropInfo ci{};
+    bool has_rows = false;
     bool ok = true;
     const uint32_t slab_bytes = (a.feat_bf16 ? 2 : 4) * kPlaneBytes;
     const int nplanes = a.feat_bf16 ? 2 : 4, plane_ch = a.feat_bf16 ? 64 : 32;
-    for (unsigned long long u = ubeg; u < uend && ok; ++u) {
-      const int b = static_cast<int>(u / nU), j = static_cast<int>(u % nU);
-      if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
-      if (ci.n == 0) continue;
+    for (uint32_t u = ubeg; u < uend && ok; ++u) {
+      const int b = static_cast<int>(u / nU32), j = static_cast<int>(u % nU32);
+      if (b != cur_b) { has_rows = crop_has_rows(a, b, lane); cur_b = b; }
+      if (!has_rows) continue;
       const int vb = j / ncb, ub = j % ncb;
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
-        if (it >= kSlabStages && !mbar_wait_bounded(&ctl->sempty[st], ph ^ 1, lim, abortp)) {
+        const bool okw = it < kSlabStages || mbar_wait_bounded(&ctl->sempty[st], ph ^ 1, lim, abortp);
+        if (!__all_sync(0xffffffffu, okw)) {
           if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
           ok = false;
           break;
@@ -455,23 +567,24 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
-    for (unsigned long long u = ubeg; u < uend && ok; ++u) {
-      const int b = static_cast<int>(u / nU);
-      if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
+    for (uint32_t u = ubeg; u < uend && ok; ++u) {
+      const int b = static_cast<int>(u / nU32);
+      if (b != cur_b) { ci = crop_info(a, b, lane, a.dec_keys != nullptr); cur_b = b; }
       if (ci.n == 0) continue;
       const int bk = a.kern_shared ? 0 : b;
       const uint32_t bytes = 2 * (ci.len0 + ci.len1) * 128;
       const CUtensorMap* km0 = ci.len0 ? &a.tmap_kern[(ci.len0 >> 3) - 1] : nullptr;
       const CUtensorMap* km1 = ci.len1 ? &a.tmap_kern[(ci.len1 >> 3) - 1] : nullptr;
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
-        if (it >= kStages && !mbar_wait_bounded(&ctl->empty[st], ph ^ 1, lim, abortp)) {
+        const bool okw = it < kStages || mbar_wait_bounded(&ctl->empty[st], ph ^ 1, lim, abortp);
+        if (!__all_sync(0xffffffffu, okw)) {
           if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
           ok = false;
           break;
         }
         if (lane == 0) {
           uint8_t* bp = bring + st * kBBytes;
-          uint64_t* fb = &ctl->ready[st];
+          uint64_t* fb = &ctl->bfull[st];
           mbar_arrive_expect_tx(fb, bytes);
           const int c0 = ch * kChunk;
 #pragma unroll
@@ -488,9 +601,9 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     if (lane == 0) {
       for (uint32_t k = 0; k < kStages && k < it; ++k) {
         const uint32_t last = it - 1 - k;
-        // the stage's phase also needs the producers: on an aborted run it may not
-        // complete, and this bounded wait then only delays the exit
-        if (!mbar_wait_drain(&ctl->ready[last % kStages], (last / kStages) & 1, lim)) atomicOr(a.err, kErrTimeout);
+        // bfull[] completes on this warp's own bytes alone, so the drain ends as
+        // soon as its copies have landed, aborted run or not
+        if (!mbar_wait_drain(&ctl->bfull[last % kStages], (last / kStages) & 1, lim)) atomicOr(a.err, kErrTimeout);
       }
     }
     __syncwarp();
@@ -506,8 +619,8 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       const uint64_t bdesc0 = make_bdesc(smem_u32(bring));
       int cur_b = -1, n = 0;
       bool ok = true;
-      for (unsigned long long u = ubeg; u < uend && ok; ++u) {
-        const int b = static_cast<int>(u / nU);
+      for (uint32_t u = ubeg; u < uend && ok; ++u) {
+        const int b = static_cast<int>(u / nU32);
         if (b != cur_b) { n = crop_n_serial(a, b); cur_b = b; }
         if (n == 0) continue;
         const uint32_t idesc = make_idesc(n);
@@ -525,7 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
         tc_fence_after();
         for (int ch = 0; ch < nchunks; ++ch, ++it) {
           GKD_TR(4, it);
-          if (!mbar_wait_bounded(&ctl->ready[st], ph, lim, abortp)) {
+          if (!mbar_wait_bounded(&ctl->bfull[st], ph, lim, abortp) ||
+              !mbar_wait_bounded(&ctl->ready[st], ph, lim, abortp)) {
             set_abort(ctl, a.err, kErrTimeout);
             ok = false;
             break;
@@ -575,12 +689,15 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
-    for (unsigned long long u = ubeg; u < uend && ok; ++u) {
-      const int b = static_cast<int>(u / nU), j = static_cast<int>(u % nU);
-      if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
+    for (uint32_t u = ubeg; u < uend && ok; ++u) {
+      const int b = static_cast<int>(u / nU32), j = static_cast<int>(u % nU32);
+      if (b != cur_b) { ci = crop_info(a, b, lane, a.dec_keys != nullptr); cur_b = b; }
       if (ci.n == 0) continue;
       const int buf = v & 1;
-      if (!mbar_wait_bounded(&ctl->accfull[buf], (v >> 1) & 1, lim, abortp)) {
+      // one decision for all four epilogue warps: they meet at named barriers below
+      const bool okw = named_bar_and(kEpiBarrier, kNumEpiWarps * 32,
+                                     mbar_wait_bounded(&ctl->accfull[buf], (v >> 1) & 1, lim, abortp));
+      if (!okw) {
         if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
         ok = false;
         break;
@@ -588,16 +705,55 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       tc_fence_after();
       if (lane == 0 && warp == kWarpEpi0) GKD_TR(9, v);
       const int Y0 = kUnitRows * (j / ncb) - 2, X0 = kUnitCols * (j % ncb);
+      if (a.dec_keys != nullptr) {
+        // decode mode: per prompt row, the fp32 mean of the modalities present
+        // (their columns are off1 apart), then one peak key per row and tile
+        // (warp max, then atomicMax across warps and tiles); no heatmap written
+        const int Yp = Y0 + my_row, Xp = X0 + my_x;
+        const bool inside = Yp >= 0 && Yp < H && Xp < W;
+        const uint32_t pixel = inside ? static_cast<uint32_t>(Yp * W + Xp) : 0u;
+        const uint8_t* mb = crop_mask(a, b);
+        const bool has0 = ci.len0 > 0, has1 = ci.len1 > 0;
+        const int kmin = has0 ? ci.kmin0 : ci.kmin1;
+        const int len = has0 ? ci.len0 : ci.len1;
+        unsigned long long* keys = a.dec_keys + static_cast<long long>(b) * a.K + kmin;
+        for (int kk = 0; kk < len; kk += kDecCols) {
+          uint32_t v0[kDecCols] = {}, v1[kDecCols] = {};
+          if (has0) tmem_ld_32x32b_x8(tmem + lane_off + buf * kMaxN + kk, v0);
+          if (has1) tmem_ld_32x32b_x8(tmem + lane_off + buf * kMaxN + ci.off1 + kk, v1);
+          tmem_wait_ld();
+          if (kk + kDecCols >= len) {   // accumulator fully read: let the MMA reuse it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->accempty[buf]);
+          }
+          unsigned long long mine = 0;   // lane i keeps the key of row kmin + kk + i
+#pragma unroll
+          for (int i = 0; i < kDecCols; ++i) {
+            const int k = kmin + kk + i;
+            if (k >= a.K) break;
+            const bool p0 = has0 && mb[k] != 0;
+            const bool p1 = has1 && mb[a.K + k] != 0;
+            if (!p0 && !p1) continue;
+            const float f0 = __uint_as_float(v0[i]), f1 = __uint_as_float(v1[i]);
+            const float f = (p0 && p1) ? __fmul_rn(__fadd_rn(f0, f1), 0.5f) : (p0 ? f0 : f1);
+            uint32_t hi, lo;
+            peak_key(f, pixel, inside, hi, lo);
+            const unsigned long long key = warp_max_key(hi, lo);
+            if (lane == i) mine = key;
+          }
+          if (mine != 0) atomicMax(keys + kk + lane, mine);
+        }
+        if (lane == 0 && warp == kWarpEpi0) GKD_TR(10, v);
+        ++v;
+        continue;
+      }
       float* hb = a.heat + static_cast<long long>(b) * a.M * a.K * P;
       const int shift0 = ci.kmin0, shift1 = a.K + ci.kmin1 - ci.off1;
       const int ngroups = ci.n / kEpiCols;
       for (int gi = 0; gi < ngroups; ++gi) {
         const int n0 = gi * kEpiCols;
-        uint32_t word = ci.vbits[0];
-#pragma unroll
-        for (int g2 = 1; g2 < 5; ++g2)
-          if ((n0 >> 5) == g2) word = ci.vbits[g2];
-        const uint32_t bits = (word >> (n0 & 31)) & 0xFFFFu;
+        const uint32_t bits = column_bits16(a, b, ci, n0, lane);
         uint32_t vv[16];
         tmem_ld_32x32b_x16(tmem + lane_off + buf * kMaxN + n0, vv);
         tmem_wait_ld();
@@ -636,88 +792,64 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     }
   } else {
     // ---------------------------------------------------------------- upsample producers
-    const int q = warp & 3;
-    const int quarter = (warp - kWarpProd0) >> 2;  // which 16 channels of each 64-channel sub-chunk
-    const int jx = lane >> 2, cq = lane & 3;       // column within the quadrant, 4-channel group
+    const int q = warp & 3;                             // lane quadrant this warp may write
+    const int grp = (warp - kWarpProd0) / kProdGroupWarps;
+    const int jx = lane >> 2, cq = lane & 3;            // column within the quadrant, 4-channel group
     const bool skip_first = (a.debug_flags & kDbgSkipProducerArrive) != 0;
-    // slab plane pitch (in 128-byte lines)
-    const int plane_lines = a.feat_5d ? kSlabLines : kPlaneSplit / 128;
-    // this thread's 4 channels inside its plane line: fp32 planes are 32 channels
-    // (16-byte chunk = 4 channels), bf16 planes 64 channels (8-byte half of a chunk)
-    const uint32_t g16 = a.feat_bf16 ? static_cast<uint32_t>(2 * quarter + (cq >> 1)) << 4
-                                     : static_cast<uint32_t>(4 * (quarter & 1) + cq) << 4;
-    const uint32_t h8 = a.feat_bf16 ? static_cast<uint32_t>(cq & 1) << 3 : 0u;
-    uint32_t it = 0, st = 0, ph = 0, ss = 0, sph = 0;   // A-ring and slab-ring positions
+    const uint32_t plane_bytes = (a.feat_5d ? kSlabLines : kPlaneSplit / 128) * 128u;
+    const uint32_t f20 = a.feat_5d ? 1u : 0u;          // plane pitch of 20 lines shifts the swizzle row by 4
+    uint32_t it = 0;
     int cur_b = -1;
-    CropInfo ci{};
+    bool has_rows = false;
     bool ok = true;
-    for (unsigned long long u = ubeg; u < uend && ok; ++u) {
-      const int b = static_cast<int>(u / nU), j = static_cast<int>(u % nU);
-      if (b != cur_b) { ci = crop_info(a, b, lane); cur_b = b; }
-      if (ci.n == 0) continue;
+    for (uint32_t u = ubeg; u < uend && ok; ++u) {
+      const int b = static_cast<int>(u / nU32), j = static_cast<int>(u % nU32);
+      if (b != cur_b) { has_rows = crop_has_rows(a, b, lane); cur_b = b; }
+      if (!has_rows) continue;
+      // this group's first stage of the unit, if it has one
+      int ch = (grp - static_cast<int>(it % kProdGroups) + kProdGroups) % kProdGroups;
+      if (ch >= nchunks) { it += nchunks; continue; }
       const Column4 cg = column_geometry(a, j / ncb, j % ncb, q, jx);
-      // per tap and sub-chunk: byte address offset of this thread's 4 channels inside a stage
-      uint32_t toff[2][4];
+      // per tap: the tap's line inside a plane plus the swizzled 16-byte chunk of
+      // this thread's first channel group; the other groups flip chunk bits
+      uint32_t base[4];
 #pragma unroll
-      for (int hs = 0; hs < 2; ++hs) {
-        const int plane = a.feat_bf16 ? hs : 2 * hs + (quarter >> 1);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int line = plane * plane_lines + cg.L[k];
-          toff[hs][k] = (static_cast<uint32_t>(line) * 128u | (g16 ^ (static_cast<uint32_t>(line & 7) << 4))) + h8;
-        }
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t L = static_cast<uint32_t>(cg.L[k]);
+        base[k] = a.feat_bf16
+                      ? (L * 128u | (((static_cast<uint32_t>(cq) >> 1) ^ (L & 7u)) << 4)) + ((cq & 1u) << 3)
+                      : (L * 128u | ((static_cast<uint32_t>(cq) ^ (L & 7u)) << 4));
       }
-      for (int ch = 0; ch < nchunks; ++ch, ++it) {
-        if (!mbar_wait_bounded(&ctl->sfull[ss], sph, lim, abortp) ||
-            (it >= kStages && !mbar_wait_bounded(&ctl->empty[st], ph ^ 1, lim, abortp))) {
+      for (; ch < nchunks; ch += kProdGroups) {
+        const uint32_t s_it = it + ch;
+        const uint32_t st = s_it % kStages, ph = (s_it / kStages) & 1;
+        const uint32_t ss = s_it % kSlabStages, sph = (s_it / kSlabStages) & 1;
+        bool okw = mbar_wait_bounded(&ctl->sfull[ss], sph, lim, abortp);
+        if (okw && s_it >= kStages) okw = mbar_wait_bounded(&ctl->empty[st], ph ^ 1, lim, abortp);
+        if (!__all_sync(0xffffffffu, okw)) {
           if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
           ok = false;
           break;
         }
         tc_fence_after();
-        if (lane == 0 && warp == kWarpProd0) GKD_TR(6, it);
+        if (lane == 0 && warp == kWarpProd0) GKD_TR(6, s_it);
         const uint32_t sp = smem_base + ss * kSlabBytes;
-#pragma unroll
-        for (int hs = 0; hs < 2; ++hs) {
-          // o[p][r]: channel pair p (4cq, 4cq+2 of this warp's 16 channels), row r
-          uint32_t o[2][4];
-          if (!a.feat_bf16) {
-            const float4 f00 = ld_shared_f4(sp + toff[hs][0]);
-            const float4 f01 = ld_shared_f4(sp + toff[hs][1]);
-            const float4 f10 = ld_shared_f4(sp + toff[hs][2]);
-            const float4 f11 = ld_shared_f4(sp + toff[hs][3]);
-            lerp_column(make_float2(f00.x, f00.y), make_float2(f01.x, f01.y), make_float2(f10.x, f10.y),
-                        make_float2(f11.x, f11.y), cg, o[0]);
-            lerp_column(make_float2(f00.z, f00.w), make_float2(f01.z, f01.w), make_float2(f10.z, f10.w),
-                        make_float2(f11.z, f11.w), cg, o[1]);
-          } else {
-            const uint2 u00 = ld_shared_u2(sp + toff[hs][0]);
-            const uint2 u01 = ld_shared_u2(sp + toff[hs][1]);
-            const uint2 u10 = ld_shared_u2(sp + toff[hs][2]);
-            const uint2 u11 = ld_shared_u2(sp + toff[hs][3]);
-            lerp_column(bf16lo_hi(u00.x), bf16lo_hi(u01.x), bf16lo_hi(u10.x), bf16lo_hi(u11.x), cg, o[0]);
-            lerp_column(bf16lo_hi(u00.y), bf16lo_hi(u01.y), bf16lo_hi(u10.y), bf16lo_hi(u11.y), cg, o[1]);
-          }
-          const uint32_t acol = tmem + kColA + st * 64 + hs * 32 + quarter * 8;
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            // lanes (jx, jx + 8) of the 16-lane half hf = rows 2 hf, 2 hf + 1
-            const uint32_t r[4] = {o[0][2 * hf], o[1][2 * hf], o[0][2 * hf + 1], o[1][2 * hf + 1]};
-            tmem_st_16x256b_x1(acol + (static_cast<uint32_t>(32 * q + 16 * hf) << 16), r);
-          }
-        }
-        if (lane == 0 && warp == kWarpProd0) GKD_TR(7, it);
+        const uint32_t acol = tmem + kColA + st * 64 + (static_cast<uint32_t>(32 * q) << 16);
+        if (a.feat_bf16)
+          produce_stage<true>(sp, base, plane_bytes, f20, cg, acol);
+        else
+          produce_stage<false>(sp, base, plane_bytes, f20, cg, acol);
+        if (lane == 0 && warp == kWarpProd0) GKD_TR(7, s_it);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&ctl->sempty[ss]);                 // slab consumed (loads completed above)
-          if (!(skip_first && it == 0)) mbar_arrive(&ctl->ready[st]);
+          if (!(skip_first && s_it == 0)) mbar_arrive(&ctl->ready[st]);
         }
-        if (lane == 0 && warp == kWarpProd0) GKD_TR(8, it);
-        if (++st == kStages) { st = 0; ph ^= 1; }
-        if (++ss == kSlabStages) { ss = 0; sph ^= 1; }
+        if (lane == 0 && warp == kWarpProd0) GKD_TR(8, s_it);
       }
+      it += nchunks;
     }
     tmem_wait_st();
   }

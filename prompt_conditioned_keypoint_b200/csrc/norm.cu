@@ -55,6 +55,93 @@ __global__ void __launch_bounds__(256) norm_rows_kernel(const float* __restrict_
   }
 }
 
+// Modality fusion moved before the contraction (the heatmap is linear in the
+// kernel row, so the mean of a prompt row's modality heatmaps, GKD_GGUF model
+// card, Model section, Architecture and Prompts bullets, is the heatmap of the
+// mean of its normalised rows). One warp per output row (crop, k): each present
+// modality's row is normalised as in norm_rows_kernel, the present ones are
+// averaged in fp32 ((a + b) * 0.5, or the one row unchanged), and the result is
+// rounded once (to bf16) on output. out_mask[b,k] = any modality present.
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256) norm_fuse_kernel(const float* __restrict__ rows,
+                                                        const uint8_t* __restrict__ mask, long long nout, int M,
+                                                        int K, int C, float eps, void* __restrict__ out,
+                                                        uint8_t* __restrict__ out_mask) {
+  const int lane = threadIdx.x & 31;
+  const long long o = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (o >= nout) return;
+  const long long b = o / K;
+  const int k = static_cast<int>(o % K);
+  const int nq = C >> 2;
+  const float4* src0 = reinterpret_cast<const float4*>(rows + ((b * M) * K + k) * C);
+  const float4* src1 = reinterpret_cast<const float4*>(rows + ((b * M + 1) * K + k) * C);
+  const bool p0 = mask[(b * M) * K + k] != 0;
+  const bool p1 = M == 2 && mask[(b * M + 1) * K + k] != 0;
+  float s0 = 0.f, s1 = 0.f;
+  for (int i = lane; i < nq; i += 32) {
+    if (p0) {
+      const float4 v = __ldg(src0 + i);
+      s0 = fmaf(v.x, v.x, s0);
+      s0 = fmaf(v.y, v.y, s0);
+      s0 = fmaf(v.z, v.z, s0);
+      s0 = fmaf(v.w, v.w, s0);
+    }
+    if (p1) {
+      const float4 v = __ldg(src1 + i);
+      s1 = fmaf(v.x, v.x, s1);
+      s1 = fmaf(v.y, v.y, s1);
+      s1 = fmaf(v.z, v.z, s1);
+      s1 = fmaf(v.w, v.w, s1);
+    }
+  }
+#pragma unroll
+  for (int sh = 16; sh > 0; sh >>= 1) {
+    s0 += __shfl_xor_sync(0xffffffffu, s0, sh);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, sh);
+  }
+  const float d0 = fmaxf(__fsqrt_rn(s0), eps), d1 = fmaxf(__fsqrt_rn(s1), eps);
+  if (lane == 0) out_mask[o] = (p0 || p1) ? 1 : 0;
+  for (int i = lane; i < nq; i += 32) {
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p0 || p1) {
+      float4 a = f, c = f;
+      if (p0) {
+        const float4 v = __ldg(src0 + i);
+        a = make_float4(__fdiv_rn(v.x, d0), __fdiv_rn(v.y, d0), __fdiv_rn(v.z, d0), __fdiv_rn(v.w, d0));
+      }
+      if (p1) {
+        const float4 v = __ldg(src1 + i);
+        c = make_float4(__fdiv_rn(v.x, d1), __fdiv_rn(v.y, d1), __fdiv_rn(v.z, d1), __fdiv_rn(v.w, d1));
+      }
+      if (p0 && p1)
+        f = make_float4(__fmul_rn(__fadd_rn(a.x, c.x), 0.5f), __fmul_rn(__fadd_rn(a.y, c.y), 0.5f),
+                        __fmul_rn(__fadd_rn(a.z, c.z), 0.5f), __fmul_rn(__fadd_rn(a.w, c.w), 0.5f));
+      else
+        f = p0 ? a : c;
+    }
+    if (OUT_BF16) {
+      reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + o * C)[i] =
+          make_uint2(pack_bf16x2(f.x, f.y), pack_bf16x2(f.z, f.w));
+    } else {
+      reinterpret_cast<float4*>(static_cast<float*>(out) + o * C)[i] = f;
+    }
+  }
+}
+
+cudaError_t launch_norm_fuse(const float* rows, const uint8_t* mask, int Bk, int M, int K, int C, float eps,
+                             bool out_bf16, void* out, uint8_t* out_mask, cudaStream_t stream) {
+  const long long nout = static_cast<long long>(Bk) * K;
+  if (nout == 0) return cudaSuccess;
+  const long long blocks = (nout + 7) / 8;
+  if (out_bf16)
+    norm_fuse_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(rows, mask, nout, M, K, C, eps, out,
+                                                                              out_mask);
+  else
+    norm_fuse_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(rows, mask, nout, M, K, C, eps, out,
+                                                                               out_mask);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_norm(const float* rows, const uint8_t* mask, long long nrows, int C, float eps,
                         bool out_bf16, void* out, cudaStream_t stream) {
   if (nrows == 0) return cudaSuccess;

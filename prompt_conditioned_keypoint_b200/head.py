@@ -8,6 +8,15 @@ steps through the C ABI on a stream:
   gkd_heatmap             fused 4x upsample + 1x1 contraction
   gkd_fuse_decode         per-row modality fusion + peak decode
 
+or, with `fused_decode=True`, gkd_heatmap_decode in place of the last two: the
+fusion and peak decode run in the heatmap kernel's epilogue and no heatmap is
+written (a [B][K] uint64 scratch buffer carries the per-row peak keys).
+
+With `fuse_rows=True` (fusion by linearity, a variant beside the graded path)
+gkd_norm_fuse_kernels replaces gkd_norm_kernels: each prompt row's modalities
+are averaged before the contraction, and the heatmap and decode steps run with
+one modality (M = 1) over the fused rows and their mask.
+
 torch only allocates memory, owns streams and copies host buffers; every step
 of the head runs in libgkd's kernels.
 """
@@ -57,24 +66,35 @@ class HeadShape:
                          wl.support is not None, float(wl.sigma), float(wl.stride), wl.up)
 
     def launches_per_step(self) -> int:
-        return 3 + (1 if self.pooled else 0)
+        """libgkd kernels one step launches: pool (if pooled), norm, then
+        heatmap + fuse_decode, or, with the decode fused, the heatmap kernel in
+        decode mode + the key finaliser (plus a cudaMemsetAsync of the scratch,
+        which is not a kernel of this library)."""
+        return (1 if self.pooled else 0) + 1 + 2
 
 
 class GkdHead:
-    def __init__(self, shape: HeadShape, device, with_fused: bool = False):
+    def __init__(self, shape: HeadShape, device, with_fused: bool = False, fused_decode: bool = False,
+                 fuse_rows: bool = False):
         s = self.shape = shape
         d = self.device = torch.device(device)
+        self.fused_decode = fused_decode
+        self.fuse_rows = fuse_rows
+        self.Mh = 1 if fuse_rows else s.M          # modalities the contraction sees
         fdt = torch.float32 if s.feat_dtype == "f32" else torch.int16
         self.feat = torch.empty((s.B, s.h, s.w, s.C), dtype=fdt, device=d)
         self.rows = torch.zeros((s.Bk, s.M, s.K, s.C), dtype=torch.float32, device=d)
         self.mask = torch.zeros((s.Bk, s.M, s.K), dtype=torch.uint8, device=d)
         kdt = torch.float32 if s.kern_dtype == "f32" else torch.int16
-        self.khat = torch.empty((s.Bk, s.M, s.K, s.C), dtype=kdt, device=d)
+        self.khat = torch.empty((s.Bk, self.Mh, s.K, s.C), dtype=kdt, device=d)
+        self.rmask = torch.empty((s.Bk, 1, s.K), dtype=torch.uint8, device=d) if fuse_rows else None
         if s.pooled:
             self.support = torch.empty((s.B, s.h, s.w, s.C), dtype=torch.float32, device=d)
             self.kpts = torch.empty((s.B, s.K, 2), dtype=torch.float32, device=d)
             self.kmask = torch.empty((s.B, s.K), dtype=torch.uint8, device=d)
-        self.heat = torch.empty((s.B, s.M, s.K, s.H, s.W), dtype=torch.float32, device=d)
+        self.heat = None if fused_decode else torch.empty((s.B, self.Mh, s.K, s.H, s.W), dtype=torch.float32,
+                                                          device=d)
+        self.scratch = torch.empty((s.B, s.K), dtype=torch.int64, device=d) if fused_decode else None
         self.fused = torch.empty((s.B, s.K, s.H, s.W), dtype=torch.float32, device=d) if with_fused else None
         self.xy = torch.empty((s.B, s.K, 2), dtype=torch.float32, device=d)
         self.score = torch.empty((s.B, s.K), dtype=torch.float32, device=d)
@@ -125,20 +145,39 @@ class GkdHead:
 
     def norm(self, stream=None):
         s = self.shape
-        gk.gkd_norm_kernels(self.rows, self.mask, s.Bk, s.M, s.K, s.C, 1e-12, DTYPE_CODE[s.kern_dtype],
-                            self.khat, stream)
+        if self.fuse_rows:
+            gk.gkd_norm_fuse_kernels(self.rows, self.mask, s.Bk, s.M, s.K, s.C, 1e-12, DTYPE_CODE[s.kern_dtype],
+                                     self.khat, self.rmask, stream)
+        else:
+            gk.gkd_norm_kernels(self.rows, self.mask, s.Bk, s.M, s.K, s.C, 1e-12, DTYPE_CODE[s.kern_dtype],
+                                self.khat, stream)
+
+    def _contraction_operands(self):
+        """(kernel rows, mask, modalities, kernel batch stride, mask batch stride) of the heatmap step."""
+        s = self.shape
+        M = self.Mh
+        mask = self.rmask if self.fuse_rows else self.mask
+        kbs = 0 if s.shared else M * s.K * s.C
+        mbs = 0 if s.shared else M * s.K
+        return self.khat, mask, M, kbs, mbs
 
     def heatmap(self, stream=None):
         s = self.shape
-        kbs = 0 if s.shared else s.M * s.K * s.C
-        mbs = 0 if s.shared else s.M * s.K
-        gk.gkd_heatmap(self.feat, DTYPE_CODE[s.feat_dtype], s.B, s.h, s.w, s.C, s.up, self.khat,
-                       DTYPE_CODE[s.kern_dtype], kbs, self.mask, mbs, s.M, s.K, self.heat, stream)
+        kern, mask, M, kbs, mbs = self._contraction_operands()
+        gk.gkd_heatmap(self.feat, DTYPE_CODE[s.feat_dtype], s.B, s.h, s.w, s.C, s.up, kern,
+                       DTYPE_CODE[s.kern_dtype], kbs, mask, mbs, M, s.K, self.heat, stream)
+
+    def heatmap_decode(self, stream=None):
+        s = self.shape
+        kern, mask, M, kbs, mbs = self._contraction_operands()
+        gk.gkd_heatmap_decode(self.feat, DTYPE_CODE[s.feat_dtype], s.B, s.h, s.w, s.C, s.up, kern,
+                              DTYPE_CODE[s.kern_dtype], kbs, mask, mbs, M, s.K, self.scratch, self.xy,
+                              self.score, self.idx, self.valid, stream)
 
     def fuse_decode(self, stream=None):
         s = self.shape
-        mbs = 0 if s.shared else s.M * s.K
-        gk.gkd_fuse_decode(self.heat, self.mask, mbs, s.B, s.M, s.K, s.H, s.W, self.fused, self.xy, self.score,
+        _, mask, M, _, mbs = self._contraction_operands()
+        gk.gkd_fuse_decode(self.heat, mask, mbs, s.B, M, s.K, s.H, s.W, self.fused, self.xy, self.score,
                            self.idx, self.valid, stream)
 
     def forward(self, stream=None, heatmap_events=None):
@@ -150,10 +189,14 @@ class GkdHead:
         self.norm(st)
         if heatmap_events is not None:
             heatmap_events[0].record(st)
-        self.heatmap(st)
+        if self.fused_decode:
+            self.heatmap_decode(st)
+        else:
+            self.heatmap(st)
         if heatmap_events is not None:
             heatmap_events[1].record(st)
-        self.fuse_decode(st)
+        if not self.fused_decode:
+            self.fuse_decode(st)
 
     def outputs_to_host(self, dst: dict | None = None, stream=None) -> dict:
         st = stream if stream is not None else torch.cuda.current_stream(self.device)
@@ -182,8 +225,12 @@ class GkdHead:
         return self.outputs_to_host(out, st)
 
     def algorithmic_heatmap_flops(self, mask: np.ndarray) -> float:
-        """2 * R * C * P summed over crops, R = valid rows of each crop."""
+        """2 * R * C * P summed over crops, R = valid rows of each crop (with
+        fuse_rows, the prompt rows with any modality present)."""
         s = self.shape
-        rows = mask.reshape(mask.shape[0], -1).sum(axis=1).astype(np.float64)
+        m = np.asarray(mask)
+        if self.fuse_rows:
+            m = m.any(axis=1)
+        rows = m.reshape(m.shape[0], -1).sum(axis=1).astype(np.float64)
         total_rows = rows[0] * s.B if s.shared else rows.sum()
         return 2.0 * total_rows * s.C * s.H * s.W

@@ -17,7 +17,9 @@ MIS = 0x10004        # misaligned stand-in
 def test_header_declares_the_boundary():
     names = gk.declared_symbols()
     assert sorted(names) == sorted([
-        "gkd_pool_prototypes", "gkd_norm_kernels", "gkd_heatmap", "gkd_fuse_decode", "gkd_last_error",
+        "gkd_pool_prototypes", "gkd_norm_kernels", "gkd_norm_fuse_kernels", "gkd_heatmap", "gkd_heatmap_decode",
+        "gkd_heatmap_contract_first", "gkd_fuse_decode",
+        "gkd_preprocess", "gkd_roi_to_image", "gkd_last_error",
         "gkd_check_device_error", "gkd_set_wait_timeout_ms", "gkd_debug_set_flags", "gkd_version"])
 
 
@@ -55,6 +57,16 @@ def test_norm_validation():
     assert "aligned" in gk.gkd_last_error() or gk.gkd_last_error() == ""
 
 
+def test_norm_fuse_validation():
+    def nf(rows=P, mask=P, Bk=2, M=2, K=80, C=1024, eps=1e-12, odt=BF16, out=P, omask=P):
+        return _status("gkd_norm_fuse_kernels", rows, mask, Bk, M, K, C, ctypes.c_float(eps), odt, out, omask, None)
+    assert nf(M=3) == SHAPE and nf(K=0) == SHAPE and nf(C=12) == SHAPE and nf(Bk=-1) == SHAPE
+    assert nf(eps=0.0) == ARG and nf(odt=4) == ARG
+    assert nf(rows=None) == ARG and nf(omask=None) == ARG
+    assert nf(rows=MIS) == ALIGN and nf(out=MIS) == ALIGN
+    assert nf(Bk=0, rows=None, mask=None, out=None, omask=None) == OK
+
+
 def test_heatmap_validation():
     def hm(feat=P, fdt=F32, B=2, h=24, w=24, C=1024, up=4, kern=P, kdt=BF16, kbs=2 * 80 * 1024, mask=P,
            mbs=160, M=2, K=80, heat=P):
@@ -79,6 +91,47 @@ def test_heatmap_validation():
     assert hm(kbs=3) == ALIGN                           # 6 bytes is not a 16-byte multiple
     assert hm(B=0, feat=None, kern=None, mask=None, heat=None) == OK
     assert "null" in gk.gkd_last_error() or gk.gkd_last_error() == ""
+
+
+def test_heatmap_decode_validation():
+    def hd(feat=P, fdt=F32, B=2, h=24, w=24, C=1024, up=4, kern=P, kdt=BF16, kbs=2 * 80 * 1024, mask=P,
+           mbs=160, M=2, K=80, scratch=P, xy=P, score=P, idx=P, valid=P):
+        return _status("gkd_heatmap_decode", feat, fdt, B, h, w, C, up, kern, kdt, kbs, mask, mbs, M, K, scratch,
+                       xy, score, idx, valid, None)
+    # the heatmap checks apply unchanged
+    assert hd(up=2) == SHAPE and hd(fdt=BF16, kdt=F32) == DTYPE and hd(M=2, K=81) == SHAPE
+    assert hd(feat=None) == ARG and hd(feat=MIS) == ALIGN and hd(kbs=3) == ALIGN
+    # and those of the decode outputs and the scratch
+    assert hd(scratch=None) == ARG and hd(xy=None) == ARG and hd(valid=None) == ARG
+    assert hd(scratch=P + 4) == ALIGN and hd(idx=P + 2) == ALIGN
+    assert hd(scratch=P + 8) in (gk.GKD_ERR_CUDA, ARG)  # 8-byte aligned is enough: reaches the pointer query
+    assert hd(B=0, feat=None, kern=None, mask=None, scratch=None, xy=None, score=None, idx=None, valid=None) == OK
+
+
+def test_contract_first_validation():
+    def cf(feat=P, fdt=F32, B=2, h=24, w=24, C=1024, up=4, kern=P, kbs=2 * 80 * 1024, mask=P, mbs=160, M=2, K=80,
+           scratch=P, heat=P):
+        return _status("gkd_heatmap_contract_first", feat, fdt, B, h, w, C, up, kern, kbs, mask, mbs, M, K, scratch,
+                       heat, None)
+    assert cf(up=2) == SHAPE and cf(M=2, K=81) == SHAPE and cf(fdt=3) == ARG
+    assert cf(scratch=None) == ARG and cf(heat=None) == ARG
+    assert cf(heat=P + 4) == ALIGN and cf(scratch=P + 2) == ALIGN
+    assert cf(B=0, feat=None, kern=None, mask=None, scratch=None, heat=None) == OK
+
+
+def test_preprocess_and_roi_validation():
+    def pp(img=P, H=480, W=640, boxes=P, B=4, canvas=384, out=P):
+        return _status("gkd_preprocess", img, H, W, boxes, B, canvas, out, None)
+    assert pp(H=0) == SHAPE and pp(W=40000) == SHAPE and pp(B=-1) == SHAPE and pp(canvas=0) == SHAPE
+    assert pp(img=None) == ARG and pp(boxes=None) == ARG and pp(out=None) == ARG
+    assert pp(out=P + 2) == ALIGN and pp(boxes=P + 1) == ALIGN
+    assert pp(B=0, img=None, boxes=None, out=None) == OK
+
+    def roi(xy=P, boxes=P, B=4, K=80, canvas=384, out=P):
+        return _status("gkd_roi_to_image", xy, boxes, B, K, canvas, out, None)
+    assert roi(K=0) == SHAPE and roi(B=70000) == SHAPE and roi(canvas=5000) == SHAPE
+    assert roi(xy=None) == ARG and roi(out=None) == ARG and roi(xy=P + 2) == ALIGN
+    assert roi(B=0, xy=None, boxes=None, out=None) == OK
 
 
 def test_pool_validation():

@@ -6,21 +6,24 @@ valid rows are skipped by every role alike):
 
   feature-slab TMA   waits sempty[s] to reuse slab slot s, arms sfull[s] with
                      the slab's bytes (one arrival plus transaction bytes);
-  kernel-row TMA     waits empty[s] to reuse stage s, arms ready[s] with the
-                     kernel rows' bytes;
+  kernel-row TMA     waits empty[s] to reuse stage s, arms bfull[s] with the
+                     kernel rows' bytes; at exit waits bfull[] of its last
+                     stages (its own copies only);
   MMA (one thread)   per unit waits accempty[buf] before reusing accumulator
-                     buf (from the third unit on); per stage waits ready[s],
-                     issues, and commits to empty[s]; at the unit's end
-                     commits to accfull[buf]; finally commits to drain;
+                     buf (from the third unit on); per stage waits bfull[s]
+                     and ready[s], issues, and commits to empty[s]; at the
+                     unit's end commits to accfull[buf]; finally commits to
+                     drain;
   epilogue warps     per unit wait accfull[buf], then each arrives once on
                      accempty[buf];
-  producer warps     per stage wait sfull[slab slot] and (from the fourth
-                     stage on) empty[s], then each arrives once on
-                     sempty[slab slot] and ready[s].
+  producer warps     in G groups of P warps; group g takes every stage i with
+                     i % G == g: waits sfull[slab slot] and (from the fourth
+                     stage on) empty[s], then each warp of the group arrives
+                     once on sempty[slab slot] and ready[s].
 
-Barrier counts: sfull 1, sempty = producer warps, ready = 1 + producer warps,
-empty 1, accfull 1, accempty = epilogue warps, drain 1. Ring depths: 6 slab
-slots, 3 stages, 2 accumulators.
+Barrier counts: sfull 1, sempty = P, bfull 1, ready = P, empty 1, accfull 1,
+accempty = epilogue warps, drain 1. Ring depths: 6 slab slots, 3 stages, 2
+accumulators.
 
 Hardware semantics modelled: a phase completes when its pending arrival count
 and its pending transaction bytes both reach zero; a parity wait on P
@@ -67,12 +70,14 @@ class Bar:
 
 
 def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=False, skip_acc_wait=False,
-             check_waits=True):
+             check_waits=True, groups=1):
     """units: valid-row counts per unit of this CTA (0 = skipped). Returns the
     number of stages run; raises AssertionError on a protocol violation.
     `bad_reuse_parity` plants a wrong parity in the producers' reuse wait;
     `skip_acc_wait` drops the MMA's wait for a drained accumulator. With
-    `check_waits` False only the data-hazard checks at each access run."""
+    `check_waits` False only the data-hazard checks at each access run.
+    `nprod` counts the warps of one producer group; `groups` groups take the
+    stages in turn."""
     rnd = random.Random(seed)
     bars = {}
 
@@ -83,7 +88,8 @@ def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=Fal
         bar(("sfull", s), 1)
         bar(("sempty", s), nprod)
     for s in range(STAGES):
-        bar(("ready", s), 1 + nprod)
+        bar(("bfull", s), 1)
+        bar(("ready", s), nprod)
         bar(("empty", s), 1)
     for t in range(2):
         bar(("accfull", t), 1)
@@ -114,9 +120,9 @@ def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=Fal
             if it >= STAGES:
                 yield ("wait", ("empty", s), (k - 1) & 1, k)
                 yield ("access", ("empty", s), k, "kernel rows overwritten before the MMA read them")
-            yield ("tx", ("ready", s), k)
+            yield ("tx", ("bfull", s), k)
         for last in range(max(0, stages - STAGES), stages):        # drain
-            yield ("wait", ("ready", last % STAGES), (last // STAGES) & 1, last // STAGES + 1)
+            yield ("wait", ("bfull", last % STAGES), (last // STAGES) & 1, last // STAGES + 1)
 
     def mma():
         it = 0
@@ -128,8 +134,10 @@ def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=Fal
                 yield ("access", ("accempty", buf), use, "accumulator overwritten before the epilogue drained it")
             for _ in range(nchunks):
                 s, k = it % STAGES, it // STAGES
+                yield ("wait", ("bfull", s), k & 1, k + 1)
+                yield ("access", ("bfull", s), k + 1, "kernel rows read before they landed")
                 yield ("wait", ("ready", s), k & 1, k + 1)
-                yield ("access", ("ready", s), k + 1, "stage read before its operands landed")
+                yield ("access", ("ready", s), k + 1, "stage read before its A operand was written")
                 yield ("commit", ("empty", s), k)
                 it += 1
             yield ("commit", ("accfull", buf), use)
@@ -144,8 +152,8 @@ def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=Fal
             yield ("access", ("accfull", buf), use + 1, "accumulator read before its MMAs completed")
             yield ("arrive", ("accempty", buf), use)
 
-    def producer():
-        for it in range(stages):
+    def producer(g):
+        for it in range(g, stages, groups):
             ss, ks = it % SLAB, it // SLAB
             s, k = it % STAGES, it // STAGES
             yield ("wait", ("sfull", ss), ks & 1, ks + 1)
@@ -158,7 +166,7 @@ def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=Fal
 
     roles = {"tma_slab": tma_slab(), "tma_rows": tma_rows(), "mma": mma()}
     roles.update({f"epi{i}": epilogue() for i in range(nepi)})
-    roles.update({f"prod{i}": producer() for i in range(nprod)})
+    roles.update({f"prod{g}.{i}": producer(g) for g in range(groups) for i in range(nprod)})
     cur = {name: next(g, None) for name, g in roles.items()}
     # per-run role speeds, so that skewed interleavings (a slow epilogue, a fast
     # issuer) are explored too, not only evenly mixed ones
@@ -210,16 +218,34 @@ def test_protocol_random_schedules(async_bias):
     for trial in range(120):
         units = [rnd.choice([0, 16, 48, 96, 160]) for _ in range(rnd.randint(0, 9))]
         total += simulate(units, rnd.randint(1, 9), nprod=rnd.randint(1, 3), nepi=rnd.randint(1, 2),
-                          seed=trial, async_bias=async_bias)
+                          seed=trial, async_bias=async_bias, groups=rnd.choice([1, 2, 3]))
     assert total > 0
 
 
 def test_protocol_with_the_kernels_warp_counts():
-    # 16 producer warps and 4 epilogue warps, as launched; long unit runs wrap
-    # every ring many times (6 slab slots, 3 stages, 2 accumulators)
+    # 4 producer groups of 4 warps and 4 epilogue warps, as launched; long unit
+    # runs wrap every ring many times (6 slab slots, 3 stages, 2 accumulators),
+    # and unit lengths that are not multiples of the group count rotate which
+    # group starts each unit
     for trial in range(6):
         units = [0, 96, 160, 0, 48, 16, 96, 96, 160, 32]
-        simulate(units, 8, nprod=16, nepi=4, seed=trial, async_bias=0.3)
+        simulate(units, 8, nprod=4, nepi=4, seed=trial, async_bias=0.3, groups=3)
+        simulate(units, 4, nprod=4, nepi=4, seed=trial, async_bias=0.3, groups=3)
+        simulate(units, 10, nprod=4, nepi=4, seed=trial, async_bias=0.3, groups=3)
+
+
+def test_model_catches_four_producer_groups():
+    """Four groups over three A slots: a group that last built stage i - 4 can
+    find empty[i % 3] two phases short of the one it needs, and a parity wait
+    cannot tell those apart. The model reports it (this is why the kernel runs
+    three groups)."""
+    failures = 0
+    for trial in range(20):
+        try:
+            simulate([96, 48, 160, 16, 96], 8, nprod=2, nepi=1, seed=trial, async_bias=0.3, groups=4)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
 
 
 def test_model_catches_a_wrong_reuse_parity():
@@ -229,7 +255,7 @@ def test_model_catches_a_wrong_reuse_parity():
     for trial in range(20):
         with pytest.raises(AssertionError):
             simulate([96, 48, 160, 16], 6, nprod=2, nepi=1, seed=trial, async_bias=0.3,
-                     bad_reuse_parity=True)
+                     bad_reuse_parity=True, groups=1 + trial % 4)
 
 
 def test_model_catches_a_missing_accumulator_wait():
