@@ -39,6 +39,8 @@ UNIT = "crops/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+# fp32 FMA peak: 148 SMs x 128 FMA lanes x 2 FLOP x 1.965 GHz (the B200's max SM clock), in TFLOP/s
+FFMA_TFLOPS = 148 * 128 * 2 * 1.965 / 1e3
 
 
 def parse_args(argv=None):
@@ -299,7 +301,7 @@ def heatmap_roofline(shape, mask, launch_s: float, peaks: dict) -> dict:
     t_hbm = hbm / (peaks["hbm_gbs"] * 1e9)
     achieved = flops / launch_s / 1e12
     if shape.kern_dtype != "bf16":
-        peak_alu = 148 * 128 * 2 * 1.965e3 / 1e3
+        peak_alu = FFMA_TFLOPS
         t_alu = flops / (peak_alu * 1e12)
         roof = {"bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s",
                 "frac": achieved / peak_alu, "roofline_us": max(t_alu, t_hbm) * 1e6}
@@ -448,7 +450,7 @@ def variant_timings(dev, stream, launches: int, peaks: dict, cfg: int = 2) -> di
     del head, G
     torch.cuda.empty_cache()
     # pooling (FFMA-bound)
-    peak_alu = 148 * 128 * 2 * 1.965e3 / 1e3
+    peak_alu = FFMA_TFLOPS
     for pc in (1, 5):
         wp = S.make_config(pc)
         hs = HeadShape.of(wp)

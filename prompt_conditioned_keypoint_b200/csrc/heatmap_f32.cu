@@ -5,10 +5,13 @@
 // Architecture bullet). Used when the kernel rows are fp32;
 // the tensor cores' fp32-input mode (tf32) would not meet a 1e-5 relative bound.
 //
-// One CTA per (crop, 4x32-pixel tile, group of up to 32 valid rows): each
-// thread owns one pixel, forms its upsampled 32-channel slice in registers
-// (4-tap, dyadic weights) and contracts it against the row chunk staged in
-// shared memory.
+// One CTA per (crop, 4x32-pixel tile, group of up to 32 valid rows), 512
+// threads: 4 channel quarters x 128 pixels. A thread owns one pixel and every
+// fourth 32-channel chunk: it forms the pixel's upsampled slice of the chunk in
+// registers (4-tap, dyadic weights) and contracts it against the chunk's rows
+// staged in shared memory. The four partial sums of a pixel are added in
+// quarter order through shared memory at the end (a fixed order: the result
+// does not depend on scheduling).
 //
 // Decode mode (`keys` non-null): a group holds 16 prompt rows with both
 // modality slots side by side, so each thread fuses its pixel's two heatmap
@@ -19,7 +22,9 @@
 
 namespace gkd {
 
-constexpr int kF32Threads = 128;
+constexpr int kF32Pix = 128;                       // pixels per CTA (4 x 32 tile)
+constexpr int kF32Quarters = 4;                    // channel quarters per CTA
+constexpr int kF32Threads = kF32Pix * kF32Quarters;
 constexpr int kF32Rows = 32;
 constexpr int kF32Chunk = 32;
 
@@ -37,7 +42,11 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
   __shared__ int rows[256];
   __shared__ int krow[128];
   __shared__ int s_nrows;
-  __shared__ float4 ks[kF32Rows][kF32Chunk / 4];
+  extern __shared__ float4 f32_smem[];
+  // one row chunk per quarter, then the partial sums of quarters 1..3
+  float4 (*ks)[kF32Rows][kF32Chunk / 4] = reinterpret_cast<float4 (*)[kF32Rows][kF32Chunk / 4]>(f32_smem);
+  float (*red)[kF32Rows][kF32Pix] =
+      reinterpret_cast<float (*)[kF32Rows][kF32Pix]>(f32_smem + kF32Quarters * kF32Rows * (kF32Chunk / 4));
 
   const int b = blockIdx.z, rg = blockIdx.y;
   const int H = 4 * h, W = 4 * w;
@@ -70,8 +79,9 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
   if (r0 >= s_nrows) return;
   const int nr = min(kF32Rows, s_nrows - r0);
 
-  const int Y = 4 * band + (threadIdx.x >> 5);
-  const int X = 32 * cb + (threadIdx.x & 31);
+  const int px = threadIdx.x % kF32Pix, qc = threadIdx.x / kF32Pix;   // pixel, channel quarter
+  const int Y = 4 * band + (px >> 5);
+  const int X = 32 * cb + (px & 31);
   int y0, y1, x0, x1;
   float ly, lx;
   taps_f32(Y, h, y0, y1, ly);
@@ -88,15 +98,18 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
 #pragma unroll
   for (int r = 0; r < kF32Rows; ++r) acc[r] = 0.f;
 
-  for (int c0 = 0; c0 < C; c0 += kF32Chunk) {
-    // stage the row chunk: nr rows x 32 channels
-    for (int t = threadIdx.x; t < kF32Rows * (kF32Chunk / 4); t += blockDim.x) {
+  const int nchunk = (C + kF32Chunk - 1) / kF32Chunk;
+  const int nround = (nchunk + kF32Quarters - 1) / kF32Quarters;
+  for (int rd = 0; rd < nround; ++rd) {
+    const int c0 = (rd * kF32Quarters + qc) * kF32Chunk;   // this quarter's chunk (may be past C)
+    // stage the row chunk: nr rows x 32 channels, by the quarter's 128 threads
+    for (int t = px; t < kF32Rows * (kF32Chunk / 4); t += kF32Pix) {
       const int r = t / (kF32Chunk / 4), q = t % (kF32Chunk / 4);
       const int c = c0 + 4 * q;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (r < nr && c < C && rows[r0 + r] >= 0)
         v = __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(rows[r0 + r]) * C + c));
-      ks[r][q] = v;
+      ks[qc][r][q] = v;
     }
     // this pixel's upsampled channels
     float u[kF32Chunk];
@@ -122,7 +135,7 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
         float s = acc[r];
 #pragma unroll
         for (int q = 0; q < kF32Chunk / 4; ++q) {
-          const float4 kv = ks[r][q];
+          const float4 kv = ks[qc][r][q];
           s = fmaf(u[4 * q + 0], kv.x, s);
           s = fmaf(u[4 * q + 1], kv.y, s);
           s = fmaf(u[4 * q + 2], kv.z, s);
@@ -133,6 +146,17 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
     }
     __syncthreads();
   }
+  // quarter 0 adds the other quarters' partial sums, in quarter order
+  if (qc > 0) {
+#pragma unroll
+    for (int r = 0; r < kF32Rows; ++r)
+      if (r < nr) red[qc - 1][r][px] = acc[r];
+  }
+  __syncthreads();
+  if (qc > 0) return;
+#pragma unroll
+  for (int r = 0; r < kF32Rows; ++r)
+    if (r < nr) acc[r] = (acc[r] + red[0][r][px]) + (red[1][r][px] + red[2][r][px]);
 
   if (decode) {
     // fuse the two modality slots of each prompt row, then one key per row and warp
@@ -171,7 +195,12 @@ cudaError_t launch_heatmap_f32(const float* feat, int B, int h, int w, int C, co
   const int W = 4 * w;
   const int groups = keys ? (K + kF32Rows / 2 - 1) / (kF32Rows / 2) : (M * K + kF32Rows - 1) / kF32Rows;
   dim3 grid(h * ((W + 31) / 32), groups, B);
-  heatmap_f32_kernel<<<grid, kF32Threads, 0, stream>>>(feat, h, w, C, kern, kern_batch_stride, mask,
+  const size_t smem = sizeof(float4) * kF32Quarters * kF32Rows * (kF32Chunk / 4) +
+                      sizeof(float) * (kF32Quarters - 1) * kF32Rows * kF32Pix;
+  cudaError_t e = cudaFuncSetAttribute(heatmap_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  heatmap_f32_kernel<<<grid, kF32Threads, smem, stream>>>(feat, h, w, C, kern, kern_batch_stride, mask,
                                                         mask_batch_stride, M, K, heat, keys);
   return cudaGetLastError();
 }

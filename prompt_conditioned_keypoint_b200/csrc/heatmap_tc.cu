@@ -43,6 +43,7 @@ namespace tc {
 #ifdef GKD_TRACE
 __device__ unsigned long long g_trace[16][2048];
 __device__ unsigned long long g_cta[1024][4];     // per CTA: start, end (ns), units, sum of n
+__device__ unsigned long long g_entry[1024];      // per CTA: kernel entry (ns)
 #define GKD_TR(kind, idx) \
   do { if (blockIdx.x == 0 && (idx) < 2048u) g_trace[kind][idx] = global_timer_ns(); } while (0)
 #else
@@ -75,11 +76,18 @@ constexpr int kEpiBufBytes = kEpiCols * kUnitRows * kEpiStride * 4;   // 10 KB
 // to fill; a parity wait is unambiguous only if the group itself saw the
 // previous phase of both barriers, so G must not exceed kStages and must divide
 // kSlabStages.
-constexpr int kProdGroups = 3, kProdGroupWarps = 4;                 // one warp per lane quadrant
-constexpr int kNumProdWarps = kProdGroups * kProdGroupWarps, kNumEpiWarps = 4;
+#ifndef GKD_EPI_HALVES
+#define GKD_EPI_HALVES 1
+#endif
+// Epilogue: kEpiHalves sets of four warps (one per lane quadrant); set e drains
+// the accumulator's column groups e, e + kEpiHalves, ...
+constexpr int kEpiHalves = GKD_EPI_HALVES;
+static_assert(kEpiHalves == 1 || kEpiHalves == 2, "epilogue sets");
+constexpr int kProdGroups = kEpiHalves == 1 ? 3 : 2, kProdGroupWarps = 4;   // one warp per lane quadrant
+constexpr int kNumProdWarps = kProdGroups * kProdGroupWarps, kNumEpiWarps = 4 * kEpiHalves;
 constexpr int kNumWarps = 3 + kNumEpiWarps + kNumProdWarps, kThreads = kNumWarps * 32;
 constexpr int kWarpTma = 0, kWarpTmaB = 1, kWarpMma = 2, kWarpEpi0 = 3, kWarpProd0 = 3 + kNumEpiWarps;
-constexpr int kEpiBarrier = 1;                   // named barrier of the four epilogue warps
+constexpr int kEpiBarrier = 1;                   // named barriers 1, 2: one per epilogue set of four warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColA = 2 * kMaxN;            // accumulators at 0 and 160; A stages at 320 + 64 s
 static_assert(kProdGroups <= kStages && kSlabStages % kProdGroups == 0, "producer groups alias ring phases");
@@ -237,9 +245,9 @@ __device__ __forceinline__ void issue_stage(uint32_t dcol, uint64_t bdesc0, uint
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
     const int hs = t >> 2, kk = t & 3;
-    umma_ts_f16(dcol, kColA + ST * 64 + hs * 32 + kk * 8,
-                bdesc0 + static_cast<uint64_t>((ST * kBBytes + hs * kBSubBytes + kk * 32) >> 4), idesc,
-                t == 0 ? first : 1u);
+    umma_ts_f16_elect(dcol, kColA + ST * 64 + hs * 32 + kk * 8,
+                      bdesc0 + static_cast<uint64_t>((ST * kBBytes + hs * kBSubBytes + kk * 32) >> 4), idesc,
+                      t == 0 ? first : 1u);
   }
 }
 
@@ -389,7 +397,7 @@ __device__ __forceinline__ void produce_stage(uint32_t sp, const uint32_t (&base
 }
 
 // ----------------------------------------------------------------------------
-__global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ HeatmapTcArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_constant__ HeatmapTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* bring = smem + kSlabStages * kSlabBytes;          // kernel-row stages
@@ -397,6 +405,9 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
   Smem* ctl = reinterpret_cast<Smem*>(epi_buf + 2 * kEpiBufBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
+#ifdef GKD_TRACE
+  if (tid == 0 && blockIdx.x < 1024) g_entry[blockIdx.x] = global_timer_ns();
+#endif
 
   const int H = 4 * a.h, W = 4 * a.w;
   const int nbands = (H + 2 + kUnitRows - 1) / kUnitRows;
@@ -449,9 +460,26 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
       }
     }
   } else {
+    // Crop sizes are found warp-cooperatively (ballots over the mask) for a chunk
+    // of kThreads crops at a time into s_cost; pass 1 sums the costs, pass 2
+    // scans them in crop order to find this CTA's first and last unit.
+    __shared__ long long s_cost[kThreads];
+    __shared__ long long s_scan[kNumWarps];
+    const bool dec = a.dec_keys != nullptr;
+    auto chunk_costs = [&](int base) {
+      for (int i = warp; i < kThreads && base + i < a.B; i += kNumWarps) {
+        const int n = crop_info(a, base + i, lane, dec).n;
+        if (lane == 0) s_cost[i] = unit_cost(n, nchunks) * nU;
+      }
+      __syncthreads();
+    };
     // pass 1: total cost
     long long local = 0;
-    for (int b = tid; b < a.B; b += kThreads) local += unit_cost(crop_n_serial(a, b), nchunks) * nU;
+    for (int base = 0; base < a.B; base += kThreads) {
+      chunk_costs(base);
+      if (base + tid < a.B) local += s_cost[tid];
+      __syncthreads();
+    }
     for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
     if (lane == 0 && local) atomicAdd(reinterpret_cast<unsigned long long*>(&ctl->total_cost),
                                       static_cast<unsigned long long>(local));
@@ -459,12 +487,12 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
     const long long T = ctl->total_cost;
     const long long tgt0 = g * T, tgt1 = (g + 1) * T;
     // pass 2: first unit whose cumulative cost before it reaches g*T/G (resp. (g+1)*T/G)
-    __shared__ long long s_scan[kNumWarps];
     long long carry = 0;
     for (int base = 0; base < a.B; base += kThreads) {
       const int b = base + tid;
-      const long long c = (b < a.B) ? unit_cost(crop_n_serial(a, b), nchunks) : 0;
-      const long long tot = c * nU;
+      if (a.B > kThreads) chunk_costs(base);           // one chunk: still in s_cost from pass 1
+      const long long tot = (b < a.B) ? s_cost[tid] : 0;
+      const long long c = tot / nU;
       long long incl = tot;
       for (int o = 1; o < 32; o <<= 1) {
         const long long v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -609,9 +637,11 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
     __syncwarp();
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA
-    // One thread runs the whole role (crop sizes computed serially, once per
-    // crop): its per-stage path is one wait, eight MMAs and one commit.
-    if (lane == 0) {
+    // The whole warp runs the role, converged: it waits, computes the crop's
+    // size and the descriptors (warp-uniform values, kept in uniform
+    // registers), and one elected lane issues each tcgen05.mma and commit. Per
+    // stage: two waits, eight MMAs, one commit.
+    {
       uint32_t it = 0, v = 0, st = 0, ph = 0;
 #ifdef GKD_TRACE
       unsigned long long trace_sum_n = 0;
@@ -621,7 +651,7 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
       bool ok = true;
       for (uint32_t u = ubeg; u < uend && ok; ++u) {
         const int b = static_cast<int>(u / nU32);
-        if (b != cur_b) { n = crop_n_serial(a, b); cur_b = b; }
+        if (b != cur_b) { n = crop_info(a, b, lane, a.dec_keys != nullptr).n; cur_b = b; }
         if (n == 0) continue;
         const uint32_t idesc = make_idesc(n);
 #ifdef GKD_TRACE
@@ -629,23 +659,25 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
 #endif
         const int buf = v & 1;
         const uint32_t dcol = buf ? kMaxN : 0u;
-        if (v >= 2 && !mbar_wait_bounded(&ctl->accempty[buf], ((v >> 1) & 1) ^ 1, lim, abortp)) {
-          set_abort(ctl, a.err, kErrTimeout);
+        const bool okw = v < 2 || mbar_wait_bounded(&ctl->accempty[buf], ((v >> 1) & 1) ^ 1, lim, abortp);
+        if (!__all_sync(0xffffffffu, okw)) {
+          if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
           ok = false;
           break;
         }
-        GKD_TR(13, v);
+        if (lane == 0) GKD_TR(13, v);
         tc_fence_after();
         for (int ch = 0; ch < nchunks; ++ch, ++it) {
-          GKD_TR(4, it);
-          if (!mbar_wait_bounded(&ctl->bfull[st], ph, lim, abortp) ||
-              !mbar_wait_bounded(&ctl->ready[st], ph, lim, abortp)) {
-            set_abort(ctl, a.err, kErrTimeout);
+          if (lane == 0) GKD_TR(4, it);
+          const bool okw2 = mbar_wait_bounded(&ctl->bfull[st], ph, lim, abortp) &&
+                            mbar_wait_bounded(&ctl->ready[st], ph, lim, abortp);
+          if (!__all_sync(0xffffffffu, okw2)) {
+            if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
             ok = false;
             break;
           }
           tc_fence_after();
-          GKD_TR(2, it);
+          if (lane == 0) GKD_TR(2, it);
           const uint32_t first = ch > 0 ? 1u : 0u;
           if (st == 0) {
             issue_stage<0>(dcol, bdesc0, idesc, first);
@@ -654,22 +686,23 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
           } else {
             issue_stage<2>(dcol, bdesc0, idesc, first);
           }
-          umma_commit(&ctl->empty[st]);
-          GKD_TR(3, it);
+          umma_commit_elect(&ctl->empty[st]);
+          if (lane == 0) GKD_TR(3, it);
           if (++st == kStages) { st = 0; ph ^= 1; }
         }
         if (!ok) break;
-        umma_commit(&ctl->accfull[buf]);
-        GKD_TR(14, v);
+        umma_commit_elect(&ctl->accfull[buf]);
+        if (lane == 0) GKD_TR(14, v);
         ++v;
       }
-      // drain: every MMA issued by this thread has completed before teardown
+      // drain: every MMA issued by this warp has completed before teardown
       if (it > 0) {
-        umma_commit(&ctl->drain);
-        if (!mbar_wait_drain(&ctl->drain, 0, lim)) atomicOr(a.err, kErrTimeout);
+        umma_commit_elect(&ctl->drain);
+        const bool drained = mbar_wait_drain(&ctl->drain, 0, lim);
+        if (lane == 0 && !drained) atomicOr(a.err, kErrTimeout);
       }
 #ifdef GKD_TRACE
-      if (blockIdx.x < 1024) {
+      if (lane == 0 && blockIdx.x < 1024) {
         g_cta[blockIdx.x][1] = global_timer_ns();
         g_cta[blockIdx.x][2] = v;
         g_cta[blockIdx.x][3] = trace_sum_n;
@@ -681,29 +714,32 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
     // ---------------------------------------------------------------- epilogue
     // TMEM -> registers -> padded shared tile [column][row][X] -> float4 rows of the heatmaps
     const int q = warp & 3;
-    const int et = tid - kWarpEpi0 * 32;           // 0..127
+    const int half = (warp - kWarpEpi0) >> 2;       // epilogue set: column groups half, half + kEpiHalves, ...
+    const int bar_id = kEpiBarrier + half;
+    const int et = tid - (kWarpEpi0 + 4 * half) * 32;   // 0..127 within the set
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
     const int my_row = 2 * (lane >> 4) + ((lane >> 3) & 1), my_x = 8 * q + (lane & 7);
-    const uint32_t epi_base = smem_u32(epi_buf);
-    uint32_t v = 0, grp = 0;
+    // one 10 KB tile per set when there are two sets, two alternating tiles for one set
+    const uint32_t epi_base = smem_u32(epi_buf) + (kEpiHalves == 2 ? half * kEpiBufBytes : 0);
+    uint32_t v = 0, grp = 0, egrp = 0;
     int cur_b = -1;
     CropInfo ci{};
     bool ok = true;
+    const bool trace_warp = warp == kWarpEpi0;
     for (uint32_t u = ubeg; u < uend && ok; ++u) {
       const int b = static_cast<int>(u / nU32), j = static_cast<int>(u % nU32);
       if (b != cur_b) { ci = crop_info(a, b, lane, a.dec_keys != nullptr); cur_b = b; }
       if (ci.n == 0) continue;
       const int buf = v & 1;
-      // one decision for all four epilogue warps: they meet at named barriers below
-      const bool okw = named_bar_and(kEpiBarrier, kNumEpiWarps * 32,
-                                     mbar_wait_bounded(&ctl->accfull[buf], (v >> 1) & 1, lim, abortp));
+      // one decision for the set's four warps: they meet at named barriers below
+      const bool okw = named_bar_and(bar_id, 128, mbar_wait_bounded(&ctl->accfull[buf], (v >> 1) & 1, lim, abortp));
       if (!okw) {
         if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
         ok = false;
         break;
       }
       tc_fence_after();
-      if (lane == 0 && warp == kWarpEpi0) GKD_TR(9, v);
+      if (lane == 0 && trace_warp) GKD_TR(9, v);
       const int Y0 = kUnitRows * (j / ncb) - 2, X0 = kUnitCols * (j % ncb);
       if (a.dec_keys != nullptr) {
         // decode mode: per prompt row, the fp32 mean of the modalities present
@@ -717,23 +753,28 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
         const int kmin = has0 ? ci.kmin0 : ci.kmin1;
         const int len = has0 ? ci.len0 : ci.len1;
         unsigned long long* keys = a.dec_keys + static_cast<long long>(b) * a.K + kmin;
-        for (int kk = 0; kk < len; kk += kDecCols) {
+        bool arrived = false;
+        for (int kk = kDecCols * half; kk < len; kk += kDecCols * kEpiHalves) {
           uint32_t v0[kDecCols] = {}, v1[kDecCols] = {};
           if (has0) tmem_ld_32x32b_x8(tmem + lane_off + buf * kMaxN + kk, v0);
           if (has1) tmem_ld_32x32b_x8(tmem + lane_off + buf * kMaxN + ci.off1 + kk, v1);
           tmem_wait_ld();
-          if (kk + kDecCols >= len) {   // accumulator fully read: let the MMA reuse it
+          if (kk + kDecCols * kEpiHalves >= len) {   // this warp's last load of the accumulator has landed
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->accempty[buf]);
+            arrived = true;
           }
+          // presence of the block's rows: bits 0-7 modality 0, bits 8-15 modality 1
+          const int kq = kmin + kk + (lane & 7);
+          const bool pres = kq < a.K && ((lane < 8 && has0 && mb[kq] != 0) ||
+                                         (lane >= 8 && lane < 16 && has1 && mb[a.K + kq] != 0));
+          const uint32_t pbits = __ballot_sync(0xffffffffu, pres);
           unsigned long long mine = 0;   // lane i keeps the key of row kmin + kk + i
 #pragma unroll
           for (int i = 0; i < kDecCols; ++i) {
-            const int k = kmin + kk + i;
-            if (k >= a.K) break;
-            const bool p0 = has0 && mb[k] != 0;
-            const bool p1 = has1 && mb[a.K + k] != 0;
+            const bool p0 = (pbits >> i) & 1u;
+            const bool p1 = (pbits >> (8 + i)) & 1u;
             if (!p0 && !p1) continue;
             const float f0 = __uint_as_float(v0[i]), f1 = __uint_as_float(v1[i]);
             const float f = (p0 && p1) ? __fmul_rn(__fadd_rn(f0, f1), 0.5f) : (p0 ? f0 : f1);
@@ -744,50 +785,84 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
           }
           if (mine != 0) atomicMax(keys + kk + lane, mine);
         }
-        if (lane == 0 && warp == kWarpEpi0) GKD_TR(10, v);
+        if (!arrived) {   // this set had no block of the accumulator
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->accempty[buf]);
+        }
+        if (lane == 0 && trace_warp) GKD_TR(10, v);
         ++v;
         continue;
       }
       float* hb = a.heat + static_cast<long long>(b) * a.M * a.K * P;
       const int shift0 = ci.kmin0, shift1 = a.K + ci.kmin1 - ci.off1;
       const int ngroups = ci.n / kEpiCols;
-      for (int gi = 0; gi < ngroups; ++gi) {
+      if (half >= ngroups) {   // no column group for this set: release the accumulator now
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->accempty[buf]);
+        ++v;
+        continue;
+      }
+      // software-pipelined: the TMEM load of the set's next group (and its
+      // validity bits) are in flight while the current group goes through
+      // shared memory to HBM
+      uint32_t cur[16], nxt[16];
+      tmem_ld_32x32b_x16(tmem + lane_off + buf * kMaxN + half * kEpiCols, cur);
+      uint32_t bits = column_bits16(a, b, ci, half * kEpiCols, lane);
+      tmem_wait_ld_regs(cur);
+      for (int gi = half; gi < ngroups; gi += kEpiHalves) {
         const int n0 = gi * kEpiCols;
-        const uint32_t bits = column_bits16(a, b, ci, n0, lane);
-        uint32_t vv[16];
-        tmem_ld_32x32b_x16(tmem + lane_off + buf * kMaxN + n0, vv);
-        tmem_wait_ld();
-        if (gi == ngroups - 1) {   // accumulator fully read: let the MMA reuse it
+        const bool more = gi + kEpiHalves < ngroups;
+        uint32_t bits_next = 0;
+        if (more) {
+          tmem_ld_32x32b_x16(tmem + lane_off + buf * kMaxN + n0 + kEpiHalves * kEpiCols, nxt);
+          bits_next = column_bits16(a, b, ci, n0 + kEpiHalves * kEpiCols, lane);
+        } else {   // every load of this accumulator by this warp has landed: let the MMA reuse it
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl->accempty[buf]);
         }
-        if (bits == 0) continue;   // uniform across the four warps (same crop)
-        // stage this thread's pixel: [col][row][X], row stride kEpiStride floats
-        const uint32_t sb = epi_base + (grp & 1) * kEpiBufBytes;
+        if (lane == 0 && trace_warp) GKD_TR(11, egrp);
+        if (bits != 0) {   // uniform across the set's four warps (same crop)
+          const uint32_t sb = epi_base + (kEpiHalves == 1 ? (grp & 1) * kEpiBufBytes : 0);
+          // one tile per set: wait until every warp of the set has read the previous group
+          if (kEpiHalves == 2 && grp > 0) named_bar_sync(bar_id, 128);
+          // stage this thread's pixel: [col][row][X], row stride kEpiStride floats
 #pragma unroll
-        for (int c = 0; c < kEpiCols; ++c)
-          st_shared_f32(sb + ((c * kUnitRows + my_row) * kEpiStride + my_x) * 4, vv[c]);
-        named_bar_sync(kEpiBarrier, kNumEpiWarps * 32);
-        // each thread writes 4 float4 (4 consecutive X of one column and row)
+          for (int c = 0; c < kEpiCols; ++c)
+            st_shared_f32(sb + ((c * kUnitRows + my_row) * kEpiStride + my_x) * 4, cur[c]);
+          named_bar_sync(bar_id, 128);
+          if (lane == 0 && trace_warp) GKD_TR(12, egrp);
+          // each thread writes 4 float4 (4 consecutive X of one column and row)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int f = i * 128 + et;
-          const int c = f >> 5, r = (f >> 3) & 3, x4 = f & 7;
-          if ((bits >> c) & 1u) {
-            const int Y = Y0 + r, X = X0 + 4 * x4;
-            if (Y >= 0 && Y < H && X < W) {
-              const float4 val = ld_shared_f4(sb + ((c * kUnitRows + r) * kEpiStride + 4 * x4) * 4);
-              const int n = n0 + c;
-              const int row = n + (n < ci.off1 ? shift0 : shift1);
-              __stcs(reinterpret_cast<float4*>(hb + static_cast<long long>(row) * P + static_cast<long long>(Y) * W + X),
-                     val);
+          for (int i = 0; i < 4; ++i) {
+            const int f = i * 128 + et;
+            const int c = f >> 5, r = (f >> 3) & 3, x4 = f & 7;
+            if ((bits >> c) & 1u) {
+              const int Y = Y0 + r, X = X0 + 4 * x4;
+              if (Y >= 0 && Y < H && X < W) {
+                const float4 val = ld_shared_f4(sb + ((c * kUnitRows + r) * kEpiStride + 4 * x4) * 4);
+                const int n = n0 + c;
+                const int row = n + (n < ci.off1 ? shift0 : shift1);
+                __stcs(reinterpret_cast<float4*>(hb + static_cast<long long>(row) * P +
+                                                 static_cast<long long>(Y) * W + X),
+                       val);
+              }
             }
           }
+          ++grp;   // staging buffers alternate only between groups that passed the barrier
         }
-        ++grp;   // staging buffers alternate only between groups that passed the barrier
+        if (lane == 0 && trace_warp) GKD_TR(15, egrp);
+        ++egrp;
+        if (more) {
+          tmem_wait_ld_regs(nxt);
+#pragma unroll
+          for (int c = 0; c < kEpiCols; ++c) cur[c] = nxt[c];
+          bits = bits_next;
+        }
       }
-      if (lane == 0 && warp == kWarpEpi0) GKD_TR(10, v);
+      if (lane == 0 && trace_warp) GKD_TR(10, v);
       ++v;
     }
   } else {
@@ -832,14 +907,18 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
           break;
         }
         tc_fence_after();
-        if (lane == 0 && warp == kWarpProd0) GKD_TR(6, s_it);
+        if (lane == 0 && (warp - kWarpProd0) % kProdGroupWarps == 0) GKD_TR(6, s_it);
         const uint32_t sp = smem_base + ss * kSlabBytes;
         const uint32_t acol = tmem + kColA + st * 64 + (static_cast<uint32_t>(32 * q) << 16);
+        // opaque per stage: keeps the compiler from hoisting the 16 swizzled tap
+        // addresses of the stage out of the loop (registers it does not have)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) asm volatile("" : "+r"(base[k]));
         if (a.feat_bf16)
           produce_stage<true>(sp, base, plane_bytes, f20, cg, acol);
         else
           produce_stage<false>(sp, base, plane_bytes, f20, cg, acol);
-        if (lane == 0 && warp == kWarpProd0) GKD_TR(7, s_it);
+        if (lane == 0 && (warp - kWarpProd0) % kProdGroupWarps == 0) GKD_TR(7, s_it);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -847,7 +926,7 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
           mbar_arrive(&ctl->sempty[ss]);                 // slab consumed (loads completed above)
           if (!(skip_first && s_it == 0)) mbar_arrive(&ctl->ready[st]);
         }
-        if (lane == 0 && warp == kWarpProd0) GKD_TR(8, s_it);
+        if (lane == 0 && (warp - kWarpProd0) % kProdGroupWarps == 0) GKD_TR(8, s_it);
       }
       it += nchunks;
     }
@@ -868,6 +947,9 @@ __global__ void __maxnreg__(104) heatmap_tc_kernel(const __grid_constant__ Heatm
 #ifdef GKD_TRACE
 extern "C" __attribute__((visibility("default"))) int gkd_trace_cta(void* host) {
   return static_cast<int>(cudaMemcpyFromSymbol(host, tc::g_cta, sizeof(tc::g_cta)));
+}
+extern "C" __attribute__((visibility("default"))) int gkd_trace_entry(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, tc::g_entry, sizeof(tc::g_entry)));
 }
 extern "C" __attribute__((visibility("default"))) int gkd_trace_read(void* host, int clear) {
   cudaError_t e = cudaMemcpyFromSymbol(host, tc::g_trace, sizeof(tc::g_trace));
