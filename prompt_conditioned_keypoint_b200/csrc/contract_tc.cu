@@ -275,21 +275,33 @@ __global__ void __launch_bounds__(kThreads, 1) contract_kernel(const __grid_cons
   }
 }
 
-// heat[b,m,k] = Up(G[b,m,k]) for valid rows; one CTA per (crop, row), 4 output
-// pixels (one float4) per thread and step.
+// heat[b,m,k] = Up(G[b,m,k]) for valid rows; one CTA per (crop, row): the row's
+// source-grid map is staged in shared memory once (read in place from global
+// memory when it does not fit, STAGED = false), then every thread writes 4
+// output pixels (one float4, streaming) per step.
+template <bool STAGED>
 __global__ void __launch_bounds__(256) upsample_kernel(const float* __restrict__ G, const uint8_t* __restrict__ mask,
                                                        long long mask_bs, int M, int K, int h, int w,
                                                        float* __restrict__ heat) {
+  extern __shared__ float gsm[];                         // [h][w] when staged
   const int row = blockIdx.x, b = blockIdx.y;          // row = m * K + k
   if (!mask[static_cast<long long>(b) * mask_bs + row]) return;
   const int H = 4 * h, W = 4 * w;
   const float* g = G + (static_cast<long long>(b) * M * K + row) * h * w;
+  const float* gs = g;
+  if (STAGED) {
+    for (int e = threadIdx.x; e < h * w; e += blockDim.x) gsm[e] = __ldg(g + e);
+    __syncthreads();
+    gs = gsm;
+  }
   float* out = heat + (static_cast<long long>(b) * M * K + row) * static_cast<long long>(H) * W;
   for (int q = threadIdx.x; q < H * W / 4; q += blockDim.x) {
     const int Y = (4 * q) / W, X0 = (4 * q) % W;
     const float sy = fmaxf((static_cast<float>(Y) + 0.5f) * 0.25f - 0.5f, 0.f);
     const int i0 = static_cast<int>(sy), i1 = min(i0 + 1, h - 1);
     const float ly = sy - static_cast<float>(i0);
+    const float* r0 = gs + i0 * w;
+    const float* r1 = gs + i1 * w;
     float v[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -297,8 +309,7 @@ __global__ void __launch_bounds__(256) upsample_kernel(const float* __restrict__
       const float sx = fmaxf((static_cast<float>(X) + 0.5f) * 0.25f - 0.5f, 0.f);
       const int j0 = static_cast<int>(sx), j1 = min(j0 + 1, w - 1);
       const float lx = sx - static_cast<float>(j0);
-      const float a0 = g[i0 * w + j0], a1 = g[i0 * w + j1], b0 = g[i1 * w + j0], b1 = g[i1 * w + j1];
-      const float t0 = fmaf(lx, a1 - a0, a0), t1 = fmaf(lx, b1 - b0, b0);
+      const float t0 = fmaf(lx, r0[j1] - r0[j0], r0[j0]), t1 = fmaf(lx, r1[j1] - r1[j0], r1[j0]);
       v[e] = fmaf(ly, t1 - t0, t0);
     }
     __stcs(reinterpret_cast<float4*>(out) + q, make_float4(v[0], v[1], v[2], v[3]));
@@ -358,7 +369,18 @@ cudaError_t launch_contract_first(ContractArgs& a, const void* feat, const void*
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2(a.M * a.K, a.B);
-  cf::upsample_kernel<<<g2, 256, 0, stream>>>(a.G, a.mask, a.mask_batch_stride, a.M, a.K, a.h, a.w, heat);
+  const size_t gsmem = sizeof(float) * static_cast<size_t>(a.h) * a.w;
+  if (gsmem <= 96 * 1024) {
+    if (gsmem > 48 * 1024) {
+      e = cudaFuncSetAttribute(cf::upsample_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(gsmem));
+      if (e != cudaSuccess) return e;
+    }
+    cf::upsample_kernel<true><<<g2, 256, gsmem, stream>>>(a.G, a.mask, a.mask_batch_stride, a.M, a.K, a.h, a.w,
+                                                          heat);
+  } else {
+    cf::upsample_kernel<false><<<g2, 256, 0, stream>>>(a.G, a.mask, a.mask_batch_stride, a.M, a.K, a.h, a.w, heat);
+  }
   return cudaGetLastError();
 }
 

@@ -63,10 +63,10 @@ constexpr int kSlabBytes = 4 * kPlaneSplit;      // fp32: 4 planes; bf16: 2 plan
 constexpr int kBSubBytes = kMaxN * 128;          // kernel rows of one sub-chunk
 constexpr int kBBytes = 2 * kBSubBytes;          // 40 KB per stage, 1 KB aligned
 #ifndef GKD_STORE_REPS
-#define GKD_STORE_REPS 2
+#define GKD_STORE_REPS 1
 #endif
-constexpr int kStoreReps = GKD_STORE_REPS;       // 16x256b repetitions per producer store (2 or 4)
-static_assert(kStoreReps == 2 || kStoreReps == 4, "producer store width");
+constexpr int kStoreReps = GKD_STORE_REPS;       // 16x256b repetitions per producer store (1, 2 or 4)
+static_assert(kStoreReps == 1 || kStoreReps == 2 || kStoreReps == 4, "producer store width");
 constexpr int kEpiCols = 16;
 constexpr int kDecCols = 8;                      // prompt rows per decode-mode block (len is a multiple of 8)                     // accumulator columns per epilogue group
 constexpr int kEpiStride = 40;                   // floats per (column, row) line of the epilogue tile
@@ -77,13 +77,16 @@ constexpr int kEpiBufBytes = kEpiCols * kUnitRows * kEpiStride * 4;   // 10 KB
 // previous phase of both barriers, so G must not exceed kStages and must divide
 // kSlabStages.
 #ifndef GKD_EPI_HALVES
-#define GKD_EPI_HALVES 1
+#define GKD_EPI_HALVES 2
 #endif
 // Epilogue: kEpiHalves sets of four warps (one per lane quadrant); set e drains
 // the accumulator's column groups e, e + kEpiHalves, ...
 constexpr int kEpiHalves = GKD_EPI_HALVES;
 static_assert(kEpiHalves == 1 || kEpiHalves == 2, "epilogue sets");
-constexpr int kProdGroups = kEpiHalves == 1 ? 3 : 2, kProdGroupWarps = 4;   // one warp per lane quadrant
+#ifndef GKD_PROD_GROUPS
+#define GKD_PROD_GROUPS 3
+#endif
+constexpr int kProdGroups = GKD_PROD_GROUPS, kProdGroupWarps = 4;   // one warp per lane quadrant
 constexpr int kNumProdWarps = kProdGroups * kProdGroupWarps, kNumEpiWarps = 4 * kEpiHalves;
 constexpr int kNumWarps = 3 + kNumEpiWarps + kNumProdWarps, kThreads = kNumWarps * 32;
 constexpr int kWarpTma = 0, kWarpTmaB = 1, kWarpMma = 2, kWarpEpi0 = 3, kWarpProd0 = 3 + kNumEpiWarps;
@@ -126,20 +129,31 @@ __device__ __forceinline__ const uint8_t* crop_mask(const HeatmapTcArgs& a, int 
 __device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int lane, bool aligned) {
   CropInfo ci;
   const uint8_t* mb = crop_mask(a, b);
+  // lane l holds mask bytes 8l .. 8l+7 of the crop's [M][K] mask (M K <= 256):
+  // eight independent loads, so one memory latency per crop
+  const int total = a.M * a.K;
+  uint32_t lb = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int p = 8 * lane + i;
+    if (p < total && mb[p] != 0) lb |= 1u << i;
+  }
   int kmin[2] = {0, 0}, len[2] = {0, 0}, last_[2] = {-1, -1};
 #pragma unroll
   for (int m = 0; m < 2; ++m) {
     if (m >= a.M) continue;
+    // this lane's valid positions of modality m, as k indices
     int first = a.K, last = -1;
-    for (int kb = 0; kb < a.K; kb += 32) {
-      const int k = kb + lane;
-      const bool v = (k < a.K) && mb[m * a.K + k] != 0;
-      const unsigned bal = __ballot_sync(0xffffffffu, v);
-      if (bal) {
-        first = min(first, kb + __ffs(bal) - 1);
-        last = kb + 31 - __clz(bal);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = 8 * lane + i - m * a.K;
+      if (((lb >> i) & 1u) && k >= 0 && k < a.K) {
+        first = min(first, k);
+        last = max(last, k);
       }
     }
+    first = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<unsigned>(first)));
+    last = __reduce_max_sync(0xffffffffu, last);
     if (last >= 0) {
       kmin[m] = first;
       last_[m] = last;
@@ -161,41 +175,35 @@ __device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int
   return ci;
 }
 
-// Warp-cooperative: bit c of the result says accumulator column n0 + c (c < 16)
-// holds a valid (m, k) row of crop b.
-__device__ __forceinline__ uint32_t column_bits16(const HeatmapTcArgs& a, int b, const CropInfo& ci, int n0,
-                                                  int lane) {
+// Thread-local: accumulator columns of crop b (the count crop_info gives), one
+// crop per thread, with 16-byte mask loads where the crop's mask is aligned.
+__device__ __forceinline__ int crop_n_thread(const HeatmapTcArgs& a, int b) {
   const uint8_t* mb = crop_mask(a, b);
-  const int col = n0 + lane;
-  bool v = false;
-  if (lane < 16 && col < ci.len0 + ci.len1) {
-    const bool m1 = col >= ci.off1;
-    const int k = (m1 ? ci.kmin1 : ci.kmin0) + (col - (m1 ? ci.off1 : 0));
-    v = k < a.K && mb[(m1 ? a.K : 0) + k] != 0;
-  }
-  return __ballot_sync(0xffffffffu, v) & 0xFFFFu;
-}
-
-// Warp-cooperative: whether crop b has any valid row (all lanes get the result).
-__device__ __forceinline__ bool crop_has_rows(const HeatmapTcArgs& a, int b, int lane) {
-  const uint8_t* mb = crop_mask(a, b);
-  const int n = a.M * a.K;
-  bool any = false;
-  for (int i = lane; i < n && !any; i += 32) any = mb[i] != 0;
-  return __any_sync(0xffffffffu, any);
-}
-
-// Thread-local (no warp collectives): number of accumulator columns of a crop
-// (the same count crop_info gives).
-__device__ __forceinline__ int crop_n_serial(const HeatmapTcArgs& a, int b) {
-  const uint8_t* mb = crop_mask(a, b);
-  int first[2] = {-1, -1}, last[2] = {-1, -1};
-  for (int m = 0; m < a.M; ++m) {
-    for (int k = 0; k < a.K; ++k)
-      if (mb[m * a.K + k]) {
-        if (first[m] < 0) first[m] = k;
-        last[m] = k;
+  const int total = a.M * a.K;
+  int first[2] = {a.K, a.K}, last[2] = {-1, -1};
+  auto take = [&](int p, bool v) {
+    if (!v) return;
+    const int m = p >= a.K ? 1 : 0, k = p - m * a.K;
+    first[m] = min(first[m], k);
+    last[m] = max(last[m], k);
+  };
+  if ((reinterpret_cast<uintptr_t>(mb) & 15u) == 0 && total % 16 == 0) {
+    const uint4* mq = reinterpret_cast<const uint4*>(mb);
+    for (int q0 = 0; q0 < total / 16; q0 += 4) {
+      uint4 v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = q0 + i < total / 16 ? __ldg(mq + q0 + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t wds[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int wq = 0; wq < 4; ++wq)
+#pragma unroll
+          for (int by = 0; by < 4; ++by) take(16 * (q0 + i) + 4 * wq + by, ((wds[wq] >> (8 * by)) & 0xFFu) != 0);
       }
+    }
+  } else {
+    for (int p = 0; p < total; ++p) take(p, mb[p] != 0);
   }
   int used = 0;
   if (a.dec_keys != nullptr && last[0] >= 0 && last[1] >= 0) {
@@ -207,14 +215,51 @@ __device__ __forceinline__ int crop_n_serial(const HeatmapTcArgs& a, int b) {
   return (used + 15) & ~15;
 }
 
-// Relative cost of one unit with n accumulator columns and nchunks 128-channel
-// stages, in eighths of one epilogue column (measured on B200: a stage takes
-// about 0.77 us and the epilogue about 0.047 us per column; a unit takes
-// whichever of its stages or the draining of the previous unit's accumulator is
-// longer, plus about an eighth of its epilogue time that the draining warps
-// take from the others).
+// Warp-cooperative: bit c of word g says accumulator column 32 g + c holds a
+// valid (m, k) row of crop b; written by lane 0 to words[0 .. 4].
+__device__ __forceinline__ void column_bits(const HeatmapTcArgs& a, int b, const CropInfo& ci, int lane,
+                                            uint32_t* words) {
+  const uint8_t* mb = crop_mask(a, b);
+  bool v[5];
+#pragma unroll
+  for (int g = 0; g < 5; ++g) {
+    const int col = 32 * g + lane;
+    v[g] = false;
+    if (col < ci.len0 + ci.len1) {
+      const bool m1 = col >= ci.off1;
+      const int k = (m1 ? ci.kmin1 : ci.kmin0) + (col - (m1 ? ci.off1 : 0));
+      v[g] = k < a.K && mb[(m1 ? a.K : 0) + k] != 0;
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < 5; ++g) {
+    const uint32_t w = __ballot_sync(0xffffffffu, v[g]);
+    if (lane == 0) words[g] = w;
+  }
+  __syncwarp();
+}
+
+// Warp-cooperative: whether crop b has any valid row (all lanes get the result).
+__device__ __forceinline__ bool crop_has_rows(const HeatmapTcArgs& a, int b, int lane) {
+  const uint8_t* mb = crop_mask(a, b);
+  const int total = a.M * a.K;
+  bool any = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int p = 8 * lane + i;
+    any |= p < total && mb[p] != 0;
+  }
+  return __any_sync(0xffffffffu, any);
+}
+
+// Relative cost of one unit with n accumulator columns and S 128-channel
+// stages, fitted to per-CTA spans of the trace build (least squares over the
+// 148 CTAs of workloads 2 to 5 on B200): a unit takes about 0.6 us per stage
+// plus 0.0125 us per column while the MMA side sets the pace, and 0.046 us per
+// column when draining its accumulator takes longer (wide crops). Units of
+// 1.25 ns.
 __device__ __forceinline__ long long unit_cost(int n, int nchunks) {
-  return n == 0 ? 0 : 8 * max(16LL * nchunks, static_cast<long long>(n)) + n;
+  return n == 0 ? 0 : max(480LL * nchunks + 10LL * n, 37LL * n);
 }
 
 __device__ __forceinline__ void src_taps(int d, int n, int& i0, int& i1, float& lam) {
@@ -242,13 +287,15 @@ __device__ __forceinline__ uint64_t make_bdesc(uint32_t smem_addr) {
 // compile-time constant: the issuing thread only adds them to fixed registers.
 template <int ST>
 __device__ __forceinline__ void issue_stage(uint32_t dcol, uint64_t bdesc0, uint32_t idesc, uint32_t first) {
+  uint32_t av[8];
+  uint64_t bv[8];
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
     const int hs = t >> 2, kk = t & 3;
-    umma_ts_f16_elect(dcol, kColA + ST * 64 + hs * 32 + kk * 8,
-                      bdesc0 + static_cast<uint64_t>((ST * kBBytes + hs * kBSubBytes + kk * 32) >> 4), idesc,
-                      t == 0 ? first : 1u);
+    av[t] = kColA + ST * 64 + hs * 32 + kk * 8;
+    bv[t] = bdesc0 + static_cast<uint64_t>((ST * kBBytes + hs * kBSubBytes + kk * 32) >> 4);
   }
+  umma_ts_f16_x8_elect(dcol, av, bv, idesc, first);
 }
 
 __device__ __forceinline__ void set_abort(Smem* ctl, unsigned* err, unsigned bits) {
@@ -389,6 +436,9 @@ __device__ __forceinline__ void produce_stage(uint32_t sp, const uint32_t (&base
     if (kStoreReps == 4) {
       tmem_st_16x256b_x4(acol + col, reinterpret_cast<const uint32_t(&)[16]>(rows01));
       tmem_st_16x256b_x4(acol + (16u << 16) + col, reinterpret_cast<const uint32_t(&)[16]>(rows23));
+    } else if (kStoreReps == 1) {
+      tmem_st_16x256b_x1(acol + col, reinterpret_cast<const uint32_t(&)[4]>(rows01));
+      tmem_st_16x256b_x1(acol + (16u << 16) + col, reinterpret_cast<const uint32_t(&)[4]>(rows23));
     } else {
       tmem_st_16x256b_x2(acol + col, reinterpret_cast<const uint32_t(&)[8]>(rows01));
       tmem_st_16x256b_x2(acol + (16u << 16) + col, reinterpret_cast<const uint32_t(&)[8]>(rows23));
@@ -451,12 +501,15 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   const unsigned long long total_units = static_cast<unsigned long long>(a.B) * nU;
   if (a.kern_shared && a.mask_batch_stride == 0) {
     // every crop has the same rows: split the units evenly
-    if (tid == 0) {
-      if (crop_n_serial(a, 0) == 0) {
-        ctl->unit_begin = ctl->unit_end = 0;
-      } else {
-        ctl->unit_begin = (total_units * g + G - 1) / G;
-        ctl->unit_end = (total_units * (g + 1) + G - 1) / G;
+    if (warp == 0) {
+      const int n0 = crop_info(a, 0, lane, a.dec_keys != nullptr).n;
+      if (lane == 0) {
+        if (n0 == 0) {
+          ctl->unit_begin = ctl->unit_end = 0;
+        } else {
+          ctl->unit_begin = (total_units * g + G - 1) / G;
+          ctl->unit_end = (total_units * (g + 1) + G - 1) / G;
+        }
       }
     }
   } else {
@@ -466,11 +519,9 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     __shared__ long long s_cost[kThreads];
     __shared__ long long s_scan[kNumWarps];
     const bool dec = a.dec_keys != nullptr;
+    (void)dec;
     auto chunk_costs = [&](int base) {
-      for (int i = warp; i < kThreads && base + i < a.B; i += kNumWarps) {
-        const int n = crop_info(a, base + i, lane, dec).n;
-        if (lane == 0) s_cost[i] = unit_cost(n, nchunks) * nU;
-      }
+      if (base + tid < a.B) s_cost[tid] = unit_cost(crop_n_thread(a, base + tid), nchunks) * nU;
       __syncthreads();
     };
     // pass 1: total cost
@@ -726,9 +777,15 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     CropInfo ci{};
     bool ok = true;
     const bool trace_warp = warp == kWarpEpi0;
+    __shared__ uint32_t s_colbits[kNumEpiWarps][5];     // valid-column bits of the current crop, per warp
+    uint32_t* colbits = s_colbits[warp - kWarpEpi0];
     for (uint32_t u = ubeg; u < uend && ok; ++u) {
       const int b = static_cast<int>(u / nU32), j = static_cast<int>(u % nU32);
-      if (b != cur_b) { ci = crop_info(a, b, lane, a.dec_keys != nullptr); cur_b = b; }
+      if (b != cur_b) {
+        ci = crop_info(a, b, lane, a.dec_keys != nullptr);
+        cur_b = b;
+        if (a.dec_keys == nullptr) column_bits(a, b, ci, lane, colbits);
+      }
       if (ci.n == 0) continue;
       const int buf = v & 1;
       // one decision for the set's four warps: they meet at named barriers below
@@ -809,7 +866,8 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       // shared memory to HBM
       uint32_t cur[16], nxt[16];
       tmem_ld_32x32b_x16(tmem + lane_off + buf * kMaxN + half * kEpiCols, cur);
-      uint32_t bits = column_bits16(a, b, ci, half * kEpiCols, lane);
+      auto group_bits = [&](int n0) { return (colbits[n0 >> 5] >> (n0 & 31)) & 0xFFFFu; };
+      uint32_t bits = group_bits(half * kEpiCols);
       tmem_wait_ld_regs(cur);
       for (int gi = half; gi < ngroups; gi += kEpiHalves) {
         const int n0 = gi * kEpiCols;
@@ -817,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
         uint32_t bits_next = 0;
         if (more) {
           tmem_ld_32x32b_x16(tmem + lane_off + buf * kMaxN + n0 + kEpiHalves * kEpiCols, nxt);
-          bits_next = column_bits16(a, b, ci, n0 + kEpiHalves * kEpiCols, lane);
+          bits_next = group_bits(n0 + kEpiHalves * kEpiCols);
         } else {   // every load of this accumulator by this warp has landed: let the MMA reuse it
           tc_fence_before();
           __syncwarp();

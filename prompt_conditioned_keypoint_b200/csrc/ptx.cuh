@@ -171,6 +171,30 @@ __device__ __forceinline__ void umma_ts_f16_elect(uint32_t d_tmem, uint32_t a_tm
       : "memory");
 }
 
+// Eight MMAs (one 128-channel stage) issued by one elected lane under a single
+// elect.sync: A columns a0 + 8 t (t = 0..7, two 32-column halves of four K=16
+// steps), B descriptors b[t]; the first accumulates iff `first` is non-zero.
+__device__ __forceinline__ void umma_ts_f16_x8_elect(uint32_t d_tmem, const uint32_t (&a)[8], const uint64_t (&b)[8],
+                                                     uint32_t idesc, uint32_t first) {
+  asm volatile(
+      "{\n\t.reg .pred p, q, e;\n\t"
+      "setp.ne.b32 p, %18, 0;\n\t"
+      "setp.eq.b32 q, %18, %18;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %9, %17, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %10, %17, q;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %11, %17, q;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %12, %17, q;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %13, %17, q;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%6], %14, %17, q;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %15, %17, q;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %16, %17, q;\n\t}"
+      ::"r"(d_tmem), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]),
+        "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc),
+        "r"(first)
+      : "memory");
+}
+
 __device__ __forceinline__ void umma_commit_elect(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"

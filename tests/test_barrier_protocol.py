@@ -232,7 +232,8 @@ def test_protocol_with_the_kernels_warp_counts():
         simulate(units, 8, nprod=4, nepi=4, seed=trial, async_bias=0.3, groups=3)
         simulate(units, 4, nprod=4, nepi=4, seed=trial, async_bias=0.3, groups=3)
         simulate(units, 10, nprod=4, nepi=4, seed=trial, async_bias=0.3, groups=3)
-        # the two-set epilogue build: 8 epilogue warps, 2 producer groups
+        # two epilogue sets (8 warps) with 3 or 2 producer groups
+        simulate(units, 8, nprod=4, nepi=8, seed=trial, async_bias=0.3, groups=3)
         simulate(units, 8, nprod=4, nepi=8, seed=trial, async_bias=0.3, groups=2)
 
 

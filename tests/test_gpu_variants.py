@@ -215,6 +215,7 @@ def run_contract_first(wl, kern_bits):
     dict(seed=74, B=2, h=3, w=9, C=64, K=128, M=1, feat_dtype="bf16", valid="random"),
     dict(seed=75, B=1, h=48, w=48, C=72, K=5, M=2, feat_dtype="f32", valid="prefix"),
     dict(seed=76, B=5, h=1, w=1, C=8, K=3, M=2, feat_dtype="f32", valid="random"),
+    dict(seed=77, B=1, h=160, w=160, C=16, K=4, M=1, feat_dtype="f32", valid="all"),   # source map > 96 KB
 ], ids=lambda c: f"s{c['seed']}")
 def test_contract_first_parity(case):
     from gpu_helpers import valid_heat_rows
