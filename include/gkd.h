@@ -228,6 +228,39 @@ GKD_API gkd_status gkd_heatmap_decode(const void* feat, gkd_dtype fdt, int B, in
                                       uint8_t* valid, void* stream);
 
 /*
+ * gkd_heatmap_decode for callers that cannot give the library any device
+ * memory: everything it needs beyond its inputs and outputs lives in one
+ * statically sized buffer inside the library. This is for code that is
+ * handed only its input and output tensors and has no way to allocate (for
+ * example a plug-in or inference-server hook without a workspace, or a
+ * process that has fixed its device memory budget at start-up and may not
+ * call cudaMalloc afterwards). The paper has no counterpart: it is an
+ * interface variant of the fused decode, not a step of the method.
+ *
+ * Arguments and outputs are those of gkd_heatmap_decode without `scratch`;
+ * the outputs are the same, bit for bit.
+ *   - The peak keys live in a file-scope __device__ array of 131072 entries
+ *     (1 MiB), which every GPU that loads the library holds until the process
+ *     exits. Calls with B * K > 131072 return GKD_ERR_SHAPE and launch nothing
+ *     (use gkd_heatmap_decode with your own scratch for those).
+ *   - The first call on a device looks up that array's device address (a
+ *     symbol lookup, no allocation) with the device current; make that first
+ *     call before any stream capture.
+ *   - Each call clears the part of the array it uses, asynchronously on
+ *     `stream`, before the heatmap kernel. All calls on a device share the
+ *     array and it keeps the last call's contents: calls that overlap on the
+ *     GPU (different streams, or different host threads) race on it and give
+ *     wrong results. Serialise them.
+ *   - The call allocates and frees nothing (no cudaMalloc, cudaFree or
+ *     allocating library routine).
+ * Limits: those of gkd_heatmap, and B * K <= 131072.
+ */
+GKD_API gkd_status gkd_heatmap_decode_noalloc(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up,
+                                              const void* kern, gkd_dtype kdt, long long kern_batch_stride,
+                                              const uint8_t* mask, long long mask_batch_stride, int M, int K,
+                                              float* xy, float* score, int32_t* idx, uint8_t* valid, void* stream);
+
+/*
  * Step 5: per-row masked fusion across modalities and peak decode ([CARD]
  * Architecture bullet, masked fusion per prompt row; Prompts bullet, text and
  * visual combined row by row; Output bullet, peak mapped to ROI -1..1 plus a

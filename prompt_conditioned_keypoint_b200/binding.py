@@ -46,6 +46,7 @@ _SIGS = {
     "gkd_heatmap": [_p, _i, _i, _i, _i, _i, _i, _p, _i, _ll, _p, _ll, _i, _i, _p, _p],
     "gkd_fuse_decode": [_p, _p, _ll, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p],
     "gkd_heatmap_decode": [_p, _i, _i, _i, _i, _i, _i, _p, _i, _ll, _p, _ll, _i, _i, _p, _p, _p, _p, _p, _p],
+    "gkd_heatmap_decode_noalloc": [_p, _i, _i, _i, _i, _i, _i, _p, _i, _ll, _p, _ll, _i, _i, _p, _p, _p, _p, _p],
     "gkd_preprocess": [_p, _i, _i, _p, _i, _i, _p, _p],
     "gkd_heatmap_contract_first": [_p, _i, _i, _i, _i, _i, _i, _p, _ll, _p, _ll, _i, _i, _p, _p, _p],
     "gkd_roi_to_image": [_p, _p, _i, _i, _i, _p, _p],
@@ -145,6 +146,13 @@ def gkd_heatmap_decode(feat, fdt, B, h, w, C, up, kern, kdt, kern_batch_stride, 
     _check("gkd_heatmap_decode", lib.gkd_heatmap_decode(
         _ptr(feat), fdt, B, h, w, C, up, _ptr(kern), kdt, kern_batch_stride, _ptr(mask), mask_batch_stride,
         M, K, _ptr(scratch), _ptr(xy), _ptr(score), _ptr(idx), _ptr(valid), _stream(stream, feat)))
+
+
+def gkd_heatmap_decode_noalloc(feat, fdt, B, h, w, C, up, kern, kdt, kern_batch_stride, mask, mask_batch_stride,
+                               M, K, xy, score, idx, valid, stream=None):
+    _check("gkd_heatmap_decode_noalloc", lib.gkd_heatmap_decode_noalloc(
+        _ptr(feat), fdt, B, h, w, C, up, _ptr(kern), kdt, kern_batch_stride, _ptr(mask), mask_batch_stride,
+        M, K, _ptr(xy), _ptr(score), _ptr(idx), _ptr(valid), _stream(stream, feat)))
 
 
 def gkd_fuse_decode(heat, mask, mask_batch_stride, B, M, K, H, W, fused, xy, score, idx, valid, stream=None):

@@ -15,6 +15,12 @@ namespace {
 
 __device__ unsigned g_device_error_word;
 
+// Peak keys of gkd_heatmap_decode_noalloc: one statically sized buffer per GPU
+// that loads the library (1 MiB, held until the process exits), for callers
+// that cannot hand the library any device memory of their own.
+constexpr long long kNoAllocKeys = 131072;     // B * K at most
+__device__ __align__(256) unsigned long long g_noalloc_keys[kNoAllocKeys];
+
 thread_local std::string t_last_error;
 std::atomic<unsigned> g_wait_timeout_ms{2000};
 std::atomic<unsigned> g_debug_flags{0};
@@ -24,6 +30,7 @@ struct DeviceState {
   bool ready = false;
   unsigned* err_word = nullptr;
   int num_sms = 0;
+  unsigned long long* noalloc_keys = nullptr;   // device address of g_noalloc_keys on this device
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -88,6 +95,12 @@ gkd_status device_state(int dev, DeviceState** out) {
     if (e != cudaSuccess) return fail(GKD_ERR_CUDA, "error word lookup failed: %s", cudaGetErrorString(e));
     e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return fail(GKD_ERR_CUDA, "SM count query failed: %s", cudaGetErrorString(e));
+    // the host-side name g_noalloc_keys is only a stand-in: kernels need its
+    // address on this device, looked up once here with the device current
+    void* k = nullptr;
+    e = cudaGetSymbolAddress(&k, g_noalloc_keys);
+    if (e != cudaSuccess) return fail(GKD_ERR_CUDA, "static key buffer lookup failed: %s", cudaGetErrorString(e));
+    d.noalloc_keys = static_cast<unsigned long long*>(k);
     d.err_word = static_cast<unsigned*>(p);
     d.ready = true;
   }
@@ -463,6 +476,32 @@ gkd_status gkd_heatmap_contract_first(const void* feat, gkd_dtype fdt, int B, in
                                              &why);
   if (e != cudaSuccess && why[0]) return fail(GKD_ERR_CUDA, "contract-first heatmap: %s", why);
   return launched(e, "contract-first heatmap");
+}
+
+gkd_status gkd_heatmap_decode_noalloc(const void* feat, gkd_dtype fdt, int B, int h, int w, int C, int up,
+                                      const void* kern, gkd_dtype kdt, long long kern_batch_stride,
+                                      const uint8_t* mask, long long mask_batch_stride, int M, int K, float* xy,
+                                      float* score, int32_t* idx, uint8_t* valid, void* stream) {
+  GKD_TRY(check_heatmap_args(feat, fdt, B, h, w, C, up, kern, kdt, kern_batch_stride, mask, mask_batch_stride, M, K));
+  if (static_cast<long long>(B) * K > kNoAllocKeys)
+    return fail(GKD_ERR_SHAPE, "B*K=%lld exceeds the %lld peak keys of the static buffer (use gkd_heatmap_decode)",
+                static_cast<long long>(B) * K, kNoAllocKeys);
+  if (B == 0) return ok();
+  if (!xy || !score || !idx || !valid) return fail(GKD_ERR_ARG, "null tensor pointer");
+  if ((reinterpret_cast<uintptr_t>(xy) | reinterpret_cast<uintptr_t>(score) | reinterpret_cast<uintptr_t>(idx)) & 3u)
+    return fail(GKD_ERR_ALIGN, "xy/score/idx must be 4-byte aligned");
+  int dev = 0;
+  GKD_TRY(use_device_of(feat, "feat", &dev));
+  GKD_TRY(check_same_device(kern, "kern", dev));
+  GKD_TRY(check_same_device(mask, "mask", dev));
+  GKD_TRY(check_same_device(xy, "xy", dev));
+  GKD_TRY(check_same_device(score, "score", dev));
+  GKD_TRY(check_same_device(idx, "idx", dev));
+  GKD_TRY(check_same_device(valid, "valid", dev));
+  DeviceState* ds = nullptr;
+  GKD_TRY(device_state(dev, &ds));
+  return enqueue_heatmap_decode(dev, feat, fdt, B, h, w, C, kern, kdt, kern_batch_stride, mask, mask_batch_stride,
+                                M, K, ds->noalloc_keys, xy, score, idx, valid, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

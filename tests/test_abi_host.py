@@ -18,7 +18,7 @@ def test_header_declares_the_boundary():
     names = gk.declared_symbols()
     assert sorted(names) == sorted([
         "gkd_pool_prototypes", "gkd_norm_kernels", "gkd_norm_fuse_kernels", "gkd_heatmap", "gkd_heatmap_decode",
-        "gkd_heatmap_contract_first", "gkd_fuse_decode",
+        "gkd_heatmap_contract_first", "gkd_heatmap_decode_noalloc", "gkd_fuse_decode",
         "gkd_preprocess", "gkd_roi_to_image", "gkd_last_error",
         "gkd_check_device_error", "gkd_set_wait_timeout_ms", "gkd_debug_set_flags", "gkd_version"])
 
@@ -132,6 +132,19 @@ def test_preprocess_and_roi_validation():
     assert roi(K=0) == SHAPE and roi(B=70000) == SHAPE and roi(canvas=5000) == SHAPE
     assert roi(xy=None) == ARG and roi(out=None) == ARG and roi(xy=P + 2) == ALIGN
     assert roi(B=0, xy=None, boxes=None, out=None) == OK
+
+
+def test_heatmap_decode_noalloc_validation():
+    def hn(feat=P, fdt=F32, B=2, h=24, w=24, C=1024, up=4, kern=P, kdt=BF16, kbs=2 * 80 * 1024, mask=P,
+           mbs=160, M=2, K=80, xy=P, score=P, idx=P, valid=P):
+        return _status("gkd_heatmap_decode_noalloc", feat, fdt, B, h, w, C, up, kern, kdt, kbs, mask, mbs, M, K,
+                       xy, score, idx, valid, None)
+    assert hn(up=2) == SHAPE and hn(M=2, K=81) == SHAPE
+    # more peak keys than the static buffer holds: rejected before anything runs
+    assert hn(B=1639, K=80) == SHAPE and "131072" in gk.gkd_last_error()
+    assert hn(B=1638, K=80) in (gk.GKD_ERR_CUDA, ARG)   # 131040 keys fit: reaches the pointer query
+    assert hn(xy=None) == ARG and hn(idx=P + 2) == ALIGN
+    assert hn(B=0, feat=None, kern=None, mask=None, xy=None, score=None, idx=None, valid=None) == OK
 
 
 def test_pool_validation():
