@@ -175,46 +175,6 @@ __device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int
   return ci;
 }
 
-// Thread-local: accumulator columns of crop b (the count crop_info gives), one
-// crop per thread, with 16-byte mask loads where the crop's mask is aligned.
-__device__ __forceinline__ int crop_n_thread(const HeatmapTcArgs& a, int b) {
-  const uint8_t* mb = crop_mask(a, b);
-  const int total = a.M * a.K;
-  int first[2] = {a.K, a.K}, last[2] = {-1, -1};
-  auto take = [&](int p, bool v) {
-    if (!v) return;
-    const int m = p >= a.K ? 1 : 0, k = p - m * a.K;
-    first[m] = min(first[m], k);
-    last[m] = max(last[m], k);
-  };
-  if ((reinterpret_cast<uintptr_t>(mb) & 15u) == 0 && total % 16 == 0) {
-    const uint4* mq = reinterpret_cast<const uint4*>(mb);
-    for (int q0 = 0; q0 < total / 16; q0 += 4) {
-      uint4 v[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = q0 + i < total / 16 ? __ldg(mq + q0 + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t wds[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-        for (int wq = 0; wq < 4; ++wq)
-#pragma unroll
-          for (int by = 0; by < 4; ++by) take(16 * (q0 + i) + 4 * wq + by, ((wds[wq] >> (8 * by)) & 0xFFu) != 0);
-      }
-    }
-  } else {
-    for (int p = 0; p < total; ++p) take(p, mb[p] != 0);
-  }
-  int used = 0;
-  if (a.dec_keys != nullptr && last[0] >= 0 && last[1] >= 0) {
-    used = 2 * ((max(last[0], last[1]) - min(first[0], first[1]) + 1 + 7) & ~7);
-  } else {
-    for (int m = 0; m < 2; ++m)
-      if (last[m] >= 0) used += (last[m] - first[m] + 1 + 7) & ~7;
-  }
-  return (used + 15) & ~15;
-}
-
 // Warp-cooperative: bit c of word g says accumulator column 32 g + c holds a
 // valid (m, k) row of crop b; written by lane 0 to words[0 .. 4].
 __device__ __forceinline__ void column_bits(const HeatmapTcArgs& a, int b, const CropInfo& ci, int lane,
@@ -285,6 +245,9 @@ __device__ __forceinline__ uint64_t make_bdesc(uint32_t smem_addr) {
 // halves x four) into the accumulator at column dcol. The tensor-memory base is
 // 0 (checked after allocation), so every A address and B-descriptor offset is a
 // compile-time constant: the issuing thread only adds them to fixed registers.
+#ifndef GKD_MMA_X8
+#define GKD_MMA_X8 1
+#endif
 template <int ST>
 __device__ __forceinline__ void issue_stage(uint32_t dcol, uint64_t bdesc0, uint32_t idesc, uint32_t first) {
   uint32_t av[8];
@@ -295,7 +258,12 @@ __device__ __forceinline__ void issue_stage(uint32_t dcol, uint64_t bdesc0, uint
     av[t] = kColA + ST * 64 + hs * 32 + kk * 8;
     bv[t] = bdesc0 + static_cast<uint64_t>((ST * kBBytes + hs * kBSubBytes + kk * 32) >> 4);
   }
-  umma_ts_f16_x8_elect(dcol, av, bv, idesc, first);
+#if GKD_MMA_X8
+  umma_ts_f16_x8_elect(dcol, av, bv, idesc, first);   // one elect for the eight
+#else
+#pragma unroll
+  for (int t = 0; t < 8; ++t) umma_ts_f16_elect(dcol, av[t], bv[t], idesc, t == 0 ? first : 1u);
+#endif
 }
 
 __device__ __forceinline__ void set_abort(Smem* ctl, unsigned* err, unsigned bits) {
@@ -519,9 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     __shared__ long long s_cost[kThreads];
     __shared__ long long s_scan[kNumWarps];
     const bool dec = a.dec_keys != nullptr;
-    (void)dec;
     auto chunk_costs = [&](int base) {
-      if (base + tid < a.B) s_cost[tid] = unit_cost(crop_n_thread(a, base + tid), nchunks) * nU;
+      for (int i = warp; i < kThreads && base + i < a.B; i += kNumWarps) {
+        const int n = crop_info(a, base + i, lane, dec).n;
+        if (lane == 0) s_cost[i] = unit_cost(n, nchunks) * nU;
+      }
       __syncthreads();
     };
     // pass 1: total cost
