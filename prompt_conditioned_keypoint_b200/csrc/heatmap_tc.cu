@@ -9,28 +9,36 @@
 // N = the crop's valid prompt rows, K = channels. Operands are bf16, the sum is
 // fp32 in tensor memory.
 //
-// Persistent kernel, one CTA per SM, 19 warps, one M=128 tile (4 output rows x
-// 32 output columns, which all read the same two source rows) per work unit:
+// One CTA per SM (218 KB of shared memory, all 512 tensor-memory columns), 24
+// warps, one M=128 tile (4 output rows x 32 output columns, which all read the
+// same two source rows) per work unit:
 //   warp 0       TMA: per 128-channel stage, a 2x10-patch feature slab (128B
 //                swizzled) into a 6-deep ring; warp 1: TMA of the stage's
 //                kernel rows (the B operand, one box per modality) into a 3-deep ring;
-//   warp 2       MMA issuer (one thread): tcgen05.mma kind::f16, A from tensor
-//                memory, B from shared memory, into one of two accumulator
-//                buffers, so the next unit accumulates while the epilogue drains;
-//   warps 3-6    epilogue: tcgen05.ld of the accumulator, transpose through a
-//                padded shared tile, coalesced float4 heatmap rows;
-//   warps 7-18   upsample producers in three groups of four warps (one warp per
-//                tensor-memory lane quadrant); group g builds the A operand of
-//                every stage i with i % 3 == g, so each warp has three stage
-//                periods for its own. A thread owns one output column of four
-//                pixels (one x-lerp per source row serves all four) and 32
-//                channels of the stage, lerps in fp32 (packed f32x2), rounds to
-//                bf16 and writes the A operand straight into tensor memory, one
-//                tcgen05.st.16x256b.x4 per 64 channels and half quadrant.
-// Units are split over CTAs by a static cost-balanced partition computed in the
-// prologue. Every wait is bounded, and every role takes the outcome of a wait
-// as one decision for all of its threads; a timeout sets the device error word
-// and all roles drain their in-flight copies and MMAs and exit.
+//   warp 2       MMA issuer: tcgen05.mma kind::f16 issued by one elected lane,
+//                A from tensor memory, B from shared memory, into one of two
+//                accumulator buffers, so the next unit accumulates while the
+//                epilogue drains;
+//   warps 3-10   epilogue, two sets of four (one warp per tensor-memory lane
+//                quadrant) taking alternate 16-column groups: tcgen05.ld of the
+//                accumulator, transpose through a padded shared tile, coalesced
+//                float4 heatmap rows;
+//   warps 11-22  upsample producers in three groups of four warps (one warp per
+//                lane quadrant); group g builds the A operand of every stage i
+//                with i % 3 == g, so each warp has three stage periods for its
+//                own. A thread owns one output column of four pixels (one x-lerp
+//                per source row serves all four) and 32 channels of the stage,
+//                lerps in fp32 (packed f32x2), rounds to bf16 and writes the A
+//                operand straight into tensor memory;
+//   warp 23      unit scheduler: the grid has one CTA per unit; a running CTA
+//                does its own unit, then takes over the units of CTAs that have
+//                not started yet with cluster launch control (a cancelled CTA
+//                never runs), so the SMs balance the work among themselves as
+//                they go. It publishes each unit with its crop's row segments
+//                into an 8-slot ring that every other warp reads.
+// Every wait is bounded, and every role takes the outcome of a wait as one
+// decision for all of its threads; a timeout sets the device error word and all
+// roles drain their in-flight copies and MMAs and exit.
 #include "decode_key.cuh"
 #include "gkd_internal.h"
 #include "ptx.cuh"
@@ -88,16 +96,37 @@ static_assert(kEpiHalves == 1 || kEpiHalves == 2, "epilogue sets");
 #endif
 constexpr int kProdGroups = GKD_PROD_GROUPS, kProdGroupWarps = 4;   // one warp per lane quadrant
 constexpr int kNumProdWarps = kProdGroups * kProdGroupWarps, kNumEpiWarps = 4 * kEpiHalves;
-constexpr int kNumWarps = 3 + kNumEpiWarps + kNumProdWarps, kThreads = kNumWarps * 32;
+constexpr int kNumWarps = 4 + kNumEpiWarps + kNumProdWarps, kThreads = kNumWarps * 32;
 constexpr int kWarpTma = 0, kWarpTmaB = 1, kWarpMma = 2, kWarpEpi0 = 3, kWarpProd0 = 3 + kNumEpiWarps;
+constexpr int kWarpSched = kNumWarps - 1;        // the unit scheduler (after the producers)
+constexpr int kUnitSlots = 8;                    // published units not yet read by every other warp
 constexpr int kEpiBarrier = 1;                   // named barriers 1, 2: one per epilogue set of four warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColA = 2 * kMaxN;            // accumulators at 0 and 160; A stages at 320 + 64 s
 static_assert(kProdGroups <= kStages && kSlabStages % kProdGroups == 0, "producer groups alias ring phases");
-constexpr size_t kSmemBytes =
-    1024 + static_cast<size_t>(kSlabStages) * kSlabBytes + static_cast<size_t>(kStages) * kBBytes + 2 * kEpiBufBytes + 512;
+constexpr size_t kCtlBytes = 1024;
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kSlabStages) * kSlabBytes +
+                              static_cast<size_t>(kStages) * kBBytes + 2 * kEpiBufBytes + kCtlBytes;
+
+struct CropInfo {
+  int n;                 // accumulator columns (multiple of 16), 0 = nothing to do
+  int kmin0, kmin1, len0, len1, off1;
+};
+
+struct alignas(16) UnitInfo {   // one work unit as the scheduler publishes it
+  int b, j, last, pad0;         // crop, tile within the crop; last: no more units
+  CropInfo ci;                  // the crop's row segments
+  uint32_t colbits[5];          // bit c of word g: accumulator column 32 g + c holds a valid row
+  int pad1;
+};
+static_assert(sizeof(UnitInfo) == 64, "unit slot size");
 
 struct Smem {            // control block placed after the stage and epilogue buffers
+  uint4 clc_resp;              // cluster-launch-control response (16-byte aligned)
+  UnitInfo units[kUnitSlots];  // the unit ring
+  uint64_t ufull[kUnitSlots];  // unit published (scheduler)
+  uint64_t uempty[kUnitSlots]; // unit read by every other warp
+  uint64_t clc_bar;            // cancellation response landed
   uint64_t sfull[kSlabStages];
   uint64_t sempty[kSlabStages];
   uint64_t bfull[kStages];     // kernel rows landed (TMA bytes)
@@ -108,14 +137,8 @@ struct Smem {            // control block placed after the stage and epilogue bu
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  unsigned long long unit_begin, unit_end;
-  long long total_cost;
 };
-
-struct CropInfo {
-  int n;                 // accumulator columns (multiple of 16), 0 = nothing to do
-  int kmin0, kmin1, len0, len1, off1;
-};
+static_assert(sizeof(Smem) <= kCtlBytes, "control block");
 
 __device__ __forceinline__ const uint8_t* crop_mask(const HeatmapTcArgs& a, int b) {
   return a.mask + static_cast<long long>(b) * a.mask_batch_stride;
@@ -176,9 +199,9 @@ __device__ __forceinline__ CropInfo crop_info(const HeatmapTcArgs& a, int b, int
 }
 
 // Warp-cooperative: bit c of word g says accumulator column 32 g + c holds a
-// valid (m, k) row of crop b; written by lane 0 to words[0 .. 4].
+// valid (m, k) row of crop b (every lane gets the five words).
 __device__ __forceinline__ void column_bits(const HeatmapTcArgs& a, int b, const CropInfo& ci, int lane,
-                                            uint32_t* words) {
+                                            uint32_t (&words)[5]) {
   const uint8_t* mb = crop_mask(a, b);
   bool v[5];
 #pragma unroll
@@ -192,34 +215,7 @@ __device__ __forceinline__ void column_bits(const HeatmapTcArgs& a, int b, const
     }
   }
 #pragma unroll
-  for (int g = 0; g < 5; ++g) {
-    const uint32_t w = __ballot_sync(0xffffffffu, v[g]);
-    if (lane == 0) words[g] = w;
-  }
-  __syncwarp();
-}
-
-// Warp-cooperative: whether crop b has any valid row (all lanes get the result).
-__device__ __forceinline__ bool crop_has_rows(const HeatmapTcArgs& a, int b, int lane) {
-  const uint8_t* mb = crop_mask(a, b);
-  const int total = a.M * a.K;
-  bool any = false;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int p = 8 * lane + i;
-    any |= p < total && mb[p] != 0;
-  }
-  return __any_sync(0xffffffffu, any);
-}
-
-// Relative cost of one unit with n accumulator columns and S 128-channel
-// stages, fitted to per-CTA spans of the trace build (least squares over the
-// 148 CTAs of workloads 2 to 5 on B200): a unit takes about 0.6 us per stage
-// plus 0.0125 us per column while the MMA side sets the pace, and 0.046 us per
-// column when draining its accumulator takes longer (wide crops). Units of
-// 1.25 ns.
-__device__ __forceinline__ long long unit_cost(int n, int nchunks) {
-  return n == 0 ? 0 : max(480LL * nchunks + 10LL * n, 37LL * n);
+  for (int g = 0; g < 5; ++g) words[g] = __ballot_sync(0xffffffffu, v[g]);
 }
 
 __device__ __forceinline__ void src_taps(int d, int n, int& i0, int& i1, float& lam) {
@@ -269,6 +265,47 @@ __device__ __forceinline__ void issue_stage(uint32_t dcol, uint64_t bdesc0, uint
 __device__ __forceinline__ void set_abort(Smem* ctl, unsigned* err, unsigned bits) {
   ctl->abort_flag = 1;
   atomicOr(err, bits);
+}
+
+// Unit ring, scheduler side: once every other warp has read the slot's
+// previous unit (bounded wait, one decision for the warp), fill slot k and
+// publish it (the arrive releases the fields to the acquiring waiters).
+__device__ __forceinline__ bool unit_publish(Smem* ctl, uint32_t k, int b, int j, int last, const CropInfo& ci,
+                                             const uint32_t (&cb)[5], uint64_t lim, volatile int* abortp,
+                                             unsigned* err, int lane) {
+  const uint32_t slot = k % kUnitSlots;
+  const bool okw = k < kUnitSlots || mbar_wait_bounded(&ctl->uempty[slot], ((k / kUnitSlots) & 1) ^ 1, lim, abortp);
+  if (!__all_sync(0xffffffffu, okw)) {
+    if (lane == 0) set_abort(ctl, err, kErrTimeout);
+    return false;
+  }
+  if (lane == 0) {
+    UnitInfo& u = ctl->units[slot];
+    u.b = b;
+    u.j = j;
+    u.last = last;
+    u.ci = ci;
+#pragma unroll
+    for (int g = 0; g < 5; ++g) u.colbits[g] = cb[g];
+    mbar_arrive(&ctl->ufull[slot]);
+  }
+  __syncwarp();
+  return true;
+}
+
+// Unit ring, reader side: wait until unit k is published (bounded, one decision
+// for the warp). The caller reads what it needs from the slot, then releases it.
+__device__ __forceinline__ bool unit_wait(Smem* ctl, uint32_t k, uint64_t lim, volatile int* abortp, unsigned* err,
+                                          int lane) {
+  const bool okw = mbar_wait_bounded(&ctl->ufull[k % kUnitSlots], (k / kUnitSlots) & 1, lim, abortp);
+  if (__all_sync(0xffffffffu, okw)) return true;
+  if (lane == 0) set_abort(ctl, err, kErrTimeout);
+  return false;
+}
+
+__device__ __forceinline__ void unit_release(Smem* ctl, uint32_t k, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&ctl->uempty[k % kUnitSlots]);
 }
 
 __device__ __forceinline__ float2 f2sub(float2 b, float2 a) {   // b - a, one rounding
@@ -434,8 +471,13 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   const int nchunks = (a.C + kChunk - 1) / kChunk;
   const long long P = static_cast<long long>(H) * W;
 
-  // ---------------- prologue: barriers, TMEM, work partition ----------------
+  // ---------------- prologue: barriers, TMEM ----------------
   if (tid == 0) {
+    for (int s = 0; s < kUnitSlots; ++s) {
+      mbar_init(&ctl->ufull[s], 1);                   // the scheduler
+      mbar_init(&ctl->uempty[s], kNumWarps - 1);      // every other warp
+    }
+    mbar_init(&ctl->clc_bar, 1);
     for (int s = 0; s < kSlabStages; ++s) {
       mbar_init(&ctl->sfull[s], 1);
       mbar_init(&ctl->sempty[s], kProdGroupWarps);
@@ -451,9 +493,6 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
-    ctl->unit_begin = ~0ull;
-    ctl->unit_end = ~0ull;
-    ctl->total_cost = 0;
     fence_mbar_init();
   }
   if (warp == kWarpMma) {
@@ -464,97 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     tma_prefetch_desc(lane == 0 ? &a.tmap_feat : &a.tmap_kern[lane - 1]);
   }
   __syncthreads();
-
-  const long long G = gridDim.x, g = blockIdx.x;
-  const unsigned long long total_units = static_cast<unsigned long long>(a.B) * nU;
-  if (a.kern_shared && a.mask_batch_stride == 0) {
-    // every crop has the same rows: split the units evenly
-    if (warp == 0) {
-      const int n0 = crop_info(a, 0, lane, a.dec_keys != nullptr).n;
-      if (lane == 0) {
-        if (n0 == 0) {
-          ctl->unit_begin = ctl->unit_end = 0;
-        } else {
-          ctl->unit_begin = (total_units * g + G - 1) / G;
-          ctl->unit_end = (total_units * (g + 1) + G - 1) / G;
-        }
-      }
-    }
-  } else {
-    // Crop sizes are found warp-cooperatively (ballots over the mask) for a chunk
-    // of kThreads crops at a time into s_cost; pass 1 sums the costs, pass 2
-    // scans them in crop order to find this CTA's first and last unit.
-    __shared__ long long s_cost[kThreads];
-    __shared__ long long s_scan[kNumWarps];
-    const bool dec = a.dec_keys != nullptr;
-    auto chunk_costs = [&](int base) {
-      for (int i = warp; i < kThreads && base + i < a.B; i += kNumWarps) {
-        const int n = crop_info(a, base + i, lane, dec).n;
-        if (lane == 0) s_cost[i] = unit_cost(n, nchunks) * nU;
-      }
-      __syncthreads();
-    };
-    // pass 1: total cost
-    long long local = 0;
-    for (int base = 0; base < a.B; base += kThreads) {
-      chunk_costs(base);
-      if (base + tid < a.B) local += s_cost[tid];
-      __syncthreads();
-    }
-    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-    if (lane == 0 && local) atomicAdd(reinterpret_cast<unsigned long long*>(&ctl->total_cost),
-                                      static_cast<unsigned long long>(local));
-    __syncthreads();
-    const long long T = ctl->total_cost;
-    const long long tgt0 = g * T, tgt1 = (g + 1) * T;
-    // pass 2: first unit whose cumulative cost before it reaches g*T/G (resp. (g+1)*T/G)
-    long long carry = 0;
-    for (int base = 0; base < a.B; base += kThreads) {
-      const int b = base + tid;
-      if (a.B > kThreads) chunk_costs(base);           // one chunk: still in s_cost from pass 1
-      const long long tot = (b < a.B) ? s_cost[tid] : 0;
-      const long long c = tot / nU;
-      long long incl = tot;
-      for (int o = 1; o < 32; o <<= 1) {
-        const long long v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      if (lane == 31) s_scan[warp] = incl;
-      __syncthreads();
-      long long wbase = 0, btot = 0;
-      for (int w2 = 0; w2 < kNumWarps; ++w2) {
-        if (w2 < warp) wbase += s_scan[w2];
-        btot += s_scan[w2];
-      }
-      const long long cb = carry + wbase + incl - tot;
-      if (c > 0) {
-        const long long cg = c * G;
-        long long need = tgt0 - cb * G;
-        long long j = need <= 0 ? 0 : (need + cg - 1) / cg;
-        if (j < nU) atomicMin(&ctl->unit_begin, static_cast<unsigned long long>(b) * nU + j);
-        need = tgt1 - cb * G;
-        j = need <= 0 ? 0 : (need + cg - 1) / cg;
-        if (j < nU) atomicMin(&ctl->unit_end, static_cast<unsigned long long>(b) * nU + j);
-      }
-      carry += btot;
-      __syncthreads();
-    }
-    if (tid == 0) {
-      if (ctl->unit_begin == ~0ull) ctl->unit_begin = total_units;
-      if (ctl->unit_end == ~0ull) ctl->unit_end = total_units;
-    }
-  }
-  if (tid == 0 && ctl->tmem_base != 0) {
-    // the MMA issue path assumes the whole tensor memory starting at column 0
-    // (the only place a 512-column allocation can land); anything else: no work
-    atomicOr(a.err, kErrBounds);
-    ctl->unit_begin = ctl->unit_end = 0;
-  }
-  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   // B * nU < 2^32 for every size the boundary accepts (65535 crops x 257 x 32 units)
-  const uint32_t ubeg = static_cast<uint32_t>(ctl->unit_begin), uend = static_cast<uint32_t>(ctl->unit_end);
   const uint32_t nU32 = static_cast<uint32_t>(nU);
 #ifdef GKD_TRACE
   if (tid == 0 && blockIdx.x < 1024) g_cta[blockIdx.x][0] = global_timer_ns();
@@ -566,15 +517,16 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   if (warp == kWarpTma) {
     // ---------------------------------------------------------------- TMA: feature slabs
     uint32_t it = 0, st = 0, ph = 0;
-    int cur_b = -1;
-    bool has_rows = false;
     bool ok = true;
     const uint32_t slab_bytes = (a.feat_bf16 ? 2 : 4) * kPlaneBytes;
     const int nplanes = a.feat_bf16 ? 2 : 4, plane_ch = a.feat_bf16 ? 64 : 32;
-    for (uint32_t u = ubeg; u < uend && ok; ++u) {
-      const int b = static_cast<int>(u / nU32), j = static_cast<int>(u % nU32);
-      if (b != cur_b) { has_rows = crop_has_rows(a, b, lane); cur_b = b; }
-      if (!has_rows) continue;
+    for (uint32_t k = 0; ok; ++k) {
+      if (!unit_wait(ctl, k, lim, abortp, a.err, lane)) break;
+      const UnitInfo& ui = ctl->units[k % kUnitSlots];
+      const int b = ui.b, j = ui.j;
+      const bool last = ui.last != 0;
+      unit_release(ctl, k, lane);
+      if (last) break;
       const int vb = j / ncb, ub = j % ncb;
       for (int ch = 0; ch < nchunks; ++ch, ++it) {
         const bool okw = it < kSlabStages || mbar_wait_bounded(&ctl->sempty[st], ph ^ 1, lim, abortp);
@@ -613,13 +565,15 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
   } else if (warp == kWarpTmaB) {
     // ---------------------------------------------------------------- TMA: kernel rows (B operand)
     uint32_t it = 0, st = 0, ph = 0;
-    int cur_b = -1;
-    CropInfo ci{};
     bool ok = true;
-    for (uint32_t u = ubeg; u < uend && ok; ++u) {
-      const int b = static_cast<int>(u / nU32);
-      if (b != cur_b) { ci = crop_info(a, b, lane, a.dec_keys != nullptr); cur_b = b; }
-      if (ci.n == 0) continue;
+    for (uint32_t k = 0; ok; ++k) {
+      if (!unit_wait(ctl, k, lim, abortp, a.err, lane)) break;
+      const UnitInfo& ui = ctl->units[k % kUnitSlots];
+      const int b = ui.b;
+      const CropInfo ci = ui.ci;
+      const bool last = ui.last != 0;
+      unit_release(ctl, k, lane);
+      if (last) break;
       const int bk = a.kern_shared ? 0 : b;
       const uint32_t bytes = 2 * (ci.len0 + ci.len1) * 128;
       const CUtensorMap* km0 = ci.len0 ? &a.tmap_kern[(ci.len0 >> 3) - 1] : nullptr;
@@ -668,12 +622,17 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       unsigned long long trace_sum_n = 0;
 #endif
       const uint64_t bdesc0 = make_bdesc(smem_u32(bring));
-      int cur_b = -1, n = 0;
       bool ok = true;
-      for (uint32_t u = ubeg; u < uend && ok; ++u) {
-        const int b = static_cast<int>(u / nU32);
-        if (b != cur_b) { n = crop_info(a, b, lane, a.dec_keys != nullptr).n; cur_b = b; }
-        if (n == 0) continue;
+      for (uint32_t k = 0; ok; ++k) {
+        if (!unit_wait(ctl, k, lim, abortp, a.err, lane)) {
+          ok = false;
+          break;
+        }
+        const UnitInfo& ui = ctl->units[k % kUnitSlots];
+        const int n = ui.ci.n;
+        const bool last = ui.last != 0;
+        unit_release(ctl, k, lane);
+        if (last) break;
         const uint32_t idesc = make_idesc(n);
 #ifdef GKD_TRACE
         trace_sum_n += n;
@@ -743,20 +702,24 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     // one 10 KB tile per set when there are two sets, two alternating tiles for one set
     const uint32_t epi_base = smem_u32(epi_buf) + (kEpiHalves == 2 ? half * kEpiBufBytes : 0);
     uint32_t v = 0, grp = 0, egrp = 0;
-    int cur_b = -1;
-    CropInfo ci{};
     bool ok = true;
     const bool trace_warp = warp == kWarpEpi0;
-    __shared__ uint32_t s_colbits[kNumEpiWarps][5];     // valid-column bits of the current crop, per warp
+    __shared__ uint32_t s_colbits[kNumEpiWarps][5];     // valid-column bits of the current unit's crop, per warp
     uint32_t* colbits = s_colbits[warp - kWarpEpi0];
-    for (uint32_t u = ubeg; u < uend && ok; ++u) {
-      const int b = static_cast<int>(u / nU32), j = static_cast<int>(u % nU32);
-      if (b != cur_b) {
-        ci = crop_info(a, b, lane, a.dec_keys != nullptr);
-        cur_b = b;
-        if (a.dec_keys == nullptr) column_bits(a, b, ci, lane, colbits);
+    for (uint32_t k = 0; ok; ++k) {
+      // one decision for the set's four warps (they meet at named barriers below)
+      if (!named_bar_and(bar_id, 128,
+                         mbar_wait_bounded(&ctl->ufull[k % kUnitSlots], (k / kUnitSlots) & 1, lim, abortp))) {
+        if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
+        break;
       }
-      if (ci.n == 0) continue;
+      const UnitInfo& ui = ctl->units[k % kUnitSlots];
+      const int b = ui.b, j = ui.j;
+      const CropInfo ci = ui.ci;
+      const bool last = ui.last != 0;
+      if (lane < 5) colbits[lane] = ui.colbits[lane];
+      unit_release(ctl, k, lane);                       // its __syncwarp also publishes colbits to the warp
+      if (last) break;
       const int buf = v & 1;
       // one decision for the set's four warps: they meet at named barriers below
       const bool okw = named_bar_and(bar_id, 128, mbar_wait_bounded(&ctl->accfull[buf], (v >> 1) & 1, lim, abortp));
@@ -893,6 +856,87 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       if (lane == 0 && trace_warp) GKD_TR(10, v);
       ++v;
     }
+  } else if (warp == kWarpSched) {
+    // ---------------------------------------------------------------- unit scheduler
+    // Work comes from the hardware's CTA queue: first this CTA's own unit (its
+    // blockIdx), then, one at a time, the units of CTAs of the grid that have not
+    // started yet, taken over by cluster launch control (a cancelled CTA never
+    // runs). Units of crops without a valid row are dropped here; every other
+    // unit goes into the ring with its crop's row segments and column bits, so
+    // that no other role reads the mask. The last entry is a stop marker.
+    const bool dec = a.dec_keys != nullptr;
+    const bool same_rows = a.kern_shared && a.mask_batch_stride == 0;   // every crop has the same rows
+    uint32_t k = 0, cph = 0, item = blockIdx.x;
+    bool ok = true, pending = false, have = true;
+    if (tmem != 0) {
+      // the MMA issue path assumes the whole tensor memory from column 0 (the only
+      // place a 512-column allocation can land); anything else: no work
+      if (lane == 0) atomicOr(a.err, kErrBounds);
+      have = false;
+    }
+    auto request = [&]() {       // one cancellation request in flight at a time
+      if (lane == 0) {
+        fence_proxy_async_smem();                       // the last response was read before it is rewritten
+        mbar_arrive_expect_tx(&ctl->clc_bar, 16);
+        clc_try_cancel(&ctl->clc_resp, &ctl->clc_bar);
+      }
+      __syncwarp();
+      pending = true;
+    };
+    // 1: a CTA was cancelled (its unit is now `item`), 0: the queue is empty, -1: the wait failed
+    auto response = [&](bool drain) -> int {
+      const bool got = drain ? mbar_wait_drain(&ctl->clc_bar, cph, lim)
+                             : mbar_wait_bounded(&ctl->clc_bar, cph, lim, abortp);
+      if (!__all_sync(0xffffffffu, got)) return -1;
+      pending = false;
+      cph ^= 1;
+      uint32_t x;
+      if (!clc_query(&ctl->clc_resp, x)) return 0;
+      item = x;
+      return 1;
+    };
+    if (have) request();
+    int cur = -1;
+    CropInfo ci{};
+    uint32_t cb[5] = {0u, 0u, 0u, 0u, 0u};
+    while (have) {
+      const int b = static_cast<int>(item / nU32), j = static_cast<int>(item % nU32);
+      if ((same_rows ? 0 : b) != cur) {
+        ci = crop_info(a, b, lane, dec);
+        if (!dec) column_bits(a, b, ci, lane, cb);
+        cur = same_rows ? 0 : b;
+      }
+      if (ci.n > 0) {
+        if (!unit_publish(ctl, k, b, j, 0, ci, cb, lim, abortp, a.err, lane)) {
+          ok = false;
+          break;
+        }
+        ++k;
+      }
+      have = false;
+      if (pending) {
+        const int r = response(false);
+        if (r < 0) {
+          if (lane == 0) set_abort(ctl, a.err, kErrTimeout);
+          ok = false;
+          break;
+        }
+        if (r > 0) {
+          have = true;
+          request();
+        }
+      }
+    }
+    if (ok) ok = unit_publish(ctl, k, 0, 0, 1, ci, cb, lim, abortp, a.err, lane);
+    // A response still in flight must land before the CTA exits. After a failure
+    // the queued CTAs are taken over without doing their units, so that none of
+    // them starts only to wait out the limit again.
+    while (pending) {
+      const int r = response(true);
+      if (r < 0 && lane == 0) atomicOr(a.err, kErrTimeout);
+      if (r <= 0) break;
+      request();
+    }
   } else {
     // ---------------------------------------------------------------- upsample producers
     const int q = warp & 3;                             // lane quadrant this warp may write
@@ -902,13 +946,13 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     const uint32_t plane_bytes = (a.feat_5d ? kSlabLines : kPlaneSplit / 128) * 128u;
     const uint32_t f20 = a.feat_5d ? 1u : 0u;          // plane pitch of 20 lines shifts the swizzle row by 4
     uint32_t it = 0;
-    int cur_b = -1;
-    bool has_rows = false;
     bool ok = true;
-    for (uint32_t u = ubeg; u < uend && ok; ++u) {
-      const int b = static_cast<int>(u / nU32), j = static_cast<int>(u % nU32);
-      if (b != cur_b) { has_rows = crop_has_rows(a, b, lane); cur_b = b; }
-      if (!has_rows) continue;
+    for (uint32_t k = 0; ok; ++k) {
+      if (!unit_wait(ctl, k, lim, abortp, a.err, lane)) break;
+      const int j = ctl->units[k % kUnitSlots].j;
+      const bool last = ctl->units[k % kUnitSlots].last != 0;
+      unit_release(ctl, k, lane);
+      if (last) break;
       // this group's first stage of the unit, if it has one
       int ch = (grp - static_cast<int>(it % kProdGroups) + kProdGroups) % kProdGroups;
       if (ch >= nchunks) { it += nchunks; continue; }
@@ -1051,9 +1095,11 @@ cudaError_t launch_heatmap_tc(HeatmapTcArgs& a, const void* feat, const void* ke
   const int H = 4 * a.h, W = 4 * a.w;
   const long long nU = static_cast<long long>((H + 2 + tc::kUnitRows - 1) / tc::kUnitRows) *
                        ((W + tc::kUnitCols - 1) / tc::kUnitCols);
+  // one CTA per unit: the SMs run one CTA each and take the queued CTAs' units
+  // over (cluster launch control), so the grid is the work list
+  (void)num_sms;
   const long long units = nU * a.B;
-  const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-  tc::heatmap_tc_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(a);
+  tc::heatmap_tc_kernel<<<static_cast<unsigned>(units), tc::kThreads, tc::kSmemBytes, stream>>>(a);
   return cudaGetLastError();
 }
 

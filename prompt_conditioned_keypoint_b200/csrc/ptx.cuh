@@ -92,6 +92,41 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 }
 
 // ----------------------------------------------------------------------------
+// Cluster launch control (sm_100): ask the hardware to cancel the launch of a
+// CTA of this grid that has not started yet. The 16-byte response is written
+// to shared memory and completes `bar` with 16 transaction bytes; a cancelled
+// CTA never runs, so the requester takes over its work. After a response that
+// reports no cancellation, no further request may be made.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];"
+      ::"r"(smem_u32(resp)), "r"(smem_u32(bar)) : "memory");
+}
+
+// Decodes a response: true (and the cancelled CTA's x index) if a CTA was cancelled.
+__device__ __forceinline__ bool clc_query(const void* resp, uint32_t& ctaid_x) {
+  uint32_t ok, x;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 h;\n\t"
+      "ld.shared.b128 h, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, h;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, h;\n\t}"
+      : "=r"(ok), "=r"(x)
+      : "r"(smem_u32(resp))
+      : "memory");
+  ctaid_x = x;
+  return ok != 0;
+}
+
+// Orders this thread's earlier generic-proxy accesses of shared memory before
+// later async-proxy writes to it.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------------
 // TMA (tensor tiled loads into shared memory, completion on an mbarrier)
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {

@@ -1,8 +1,15 @@
 """CPU model of the tensor-core heatmap kernel's mbarrier protocol (no GPU).
 
-The persistent kernel in csrc/heatmap_tc.cu runs five roles per CTA over its
-range of work units (one unit = 128 output pixels of one crop; crops with no
-valid rows are skipped by every role alike):
+The kernel in csrc/heatmap_tc.cu runs six roles per CTA over the work units
+it is given (one unit = 128 output pixels of one crop):
+
+  scheduler          takes units from the hardware's CTA queue, drops those
+                     of crops with no valid row, and publishes the others into
+                     a ring of U slots: waits uempty[slot] before reusing a
+                     slot (from the (U+1)-th unit on), fills it, arrives on
+                     ufull[slot]; a stop marker follows the last unit;
+  every other warp   per unit waits ufull[slot], reads the slot, arrives once
+                     on uempty[slot] (also for the stop marker), then:
 
   feature-slab TMA   waits sempty[s] to reuse slab slot s, arms sfull[s] with
                      the slab's bytes (one arrival plus transaction bytes);
@@ -21,9 +28,9 @@ valid rows are skipped by every role alike):
                      stage on) empty[s], then each warp of the group arrives
                      once on sempty[slab slot] and ready[s].
 
-Barrier counts: sfull 1, sempty = P, bfull 1, ready = P, empty 1, accfull 1,
-accempty = epilogue warps, drain 1. Ring depths: 6 slab slots, 3 stages, 2
-accumulators.
+Barrier counts: ufull 1, uempty = every warp but the scheduler, sfull 1,
+sempty = P, bfull 1, ready = P, empty 1, accfull 1, accempty = epilogue warps,
+drain 1. Ring depths: 8 unit slots, 6 slab slots, 3 stages, 2 accumulators.
 
 Hardware semantics modelled: a phase completes when its pending arrival count
 and its pending transaction bytes both reach zero; a parity wait on P
@@ -40,7 +47,7 @@ import random
 
 import pytest
 
-SLAB, STAGES = 6, 3
+SLAB, STAGES, UNIT_SLOTS = 6, 3, 8
 
 
 class Bar:
@@ -70,14 +77,15 @@ class Bar:
 
 
 def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=False, skip_acc_wait=False,
-             check_waits=True, groups=1):
+             check_waits=True, groups=1, skip_slot_wait=False):
     """units: valid-row counts per unit of this CTA (0 = skipped). Returns the
     number of stages run; raises AssertionError on a protocol violation.
     `bad_reuse_parity` plants a wrong parity in the producers' reuse wait;
     `skip_acc_wait` drops the MMA's wait for a drained accumulator. With
     `check_waits` False only the data-hazard checks at each access run.
     `nprod` counts the warps of one producer group; `groups` groups take the
-    stages in turn."""
+    stages in turn. `skip_slot_wait` drops the scheduler's wait for a read
+    unit slot."""
     rnd = random.Random(seed)
     bars = {}
 
@@ -95,6 +103,10 @@ def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=Fal
         bar(("accfull", t), 1)
         bar(("accempty", t), nepi)
     bar(("drain",), 1)
+    nreaders = 3 + nepi + groups * nprod
+    for s in range(UNIT_SLOTS):
+        bar(("ufull", s), 1)
+        bar(("uempty", s), nreaders)
     live = [n for n in units if n > 0]
     stages = len(live) * nchunks
     tx_in_flight = []          # barriers with transaction bytes still landing
@@ -104,29 +116,59 @@ def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=Fal
     #                 | ("tx", bar, phase) | ("commit", bar, phase)
     #                 | ("access", bar, phases_needed, what): a read or overwrite of the
     #                   buffer that `bar` guards, legal once `bar` has completed that many phases
+    def scheduler():
+        for v in range(len(live) + 1):                            # the units, then the stop marker
+            s, k = v % UNIT_SLOTS, v // UNIT_SLOTS
+            if v >= UNIT_SLOTS:
+                if not skip_slot_wait:
+                    yield ("wait", ("uempty", s), (k - 1) & 1, k)
+                yield ("access", ("uempty", s), k, "unit slot overwritten before every warp read it")
+            yield ("arrive", ("ufull", s), k)
+
+    def take_unit(v):
+        s, k = v % UNIT_SLOTS, v // UNIT_SLOTS
+        yield ("wait", ("ufull", s), k & 1, k + 1)
+        yield ("access", ("ufull", s), k + 1, "unit slot read before it was published")
+        yield ("arrive", ("uempty", s), k)
+
     def tma_slab():
-        for it in range(stages):
-            s, k = it % SLAB, it // SLAB
-            if it >= SLAB:
-                yield ("wait", ("sempty", s), (k - 1) & 1, k)
-                yield ("access", ("sempty", s), k, "slab slot overwritten before the producers read it")
-            yield ("tx", ("sfull", s), k)
+        it = 0
+        for v in range(len(live) + 1):
+            yield from take_unit(v)
+            if v == len(live):
+                break
+            for _ in range(nchunks):
+                s, k = it % SLAB, it // SLAB
+                if it >= SLAB:
+                    yield ("wait", ("sempty", s), (k - 1) & 1, k)
+                    yield ("access", ("sempty", s), k, "slab slot overwritten before the producers read it")
+                yield ("tx", ("sfull", s), k)
+                it += 1
         for last in range(max(0, stages - SLAB), stages):          # drain
             yield ("wait", ("sfull", last % SLAB), (last // SLAB) & 1, last // SLAB + 1)
 
     def tma_rows():
-        for it in range(stages):
-            s, k = it % STAGES, it // STAGES
-            if it >= STAGES:
-                yield ("wait", ("empty", s), (k - 1) & 1, k)
-                yield ("access", ("empty", s), k, "kernel rows overwritten before the MMA read them")
-            yield ("tx", ("bfull", s), k)
+        it = 0
+        for v in range(len(live) + 1):
+            yield from take_unit(v)
+            if v == len(live):
+                break
+            for _ in range(nchunks):
+                s, k = it % STAGES, it // STAGES
+                if it >= STAGES:
+                    yield ("wait", ("empty", s), (k - 1) & 1, k)
+                    yield ("access", ("empty", s), k, "kernel rows overwritten before the MMA read them")
+                yield ("tx", ("bfull", s), k)
+                it += 1
         for last in range(max(0, stages - STAGES), stages):        # drain
             yield ("wait", ("bfull", last % STAGES), (last // STAGES) & 1, last // STAGES + 1)
 
     def mma():
         it = 0
-        for v in range(len(live)):
+        for v in range(len(live) + 1):
+            yield from take_unit(v)
+            if v == len(live):
+                break
             buf, use = v & 1, v >> 1
             if v >= 2 and not skip_acc_wait:
                 yield ("wait", ("accempty", buf), (use - 1) & 1, use)
@@ -146,14 +188,26 @@ def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=Fal
             yield ("wait", ("drain",), 0, 1)
 
     def epilogue():
-        for v in range(len(live)):
+        for v in range(len(live) + 1):
+            yield from take_unit(v)
+            if v == len(live):
+                break
             buf, use = v & 1, v >> 1
             yield ("wait", ("accfull", buf), use & 1, use + 1)
             yield ("access", ("accfull", buf), use + 1, "accumulator read before its MMAs completed")
             yield ("arrive", ("accempty", buf), use)
 
     def producer(g):
-        for it in range(g, stages, groups):
+        for v in range(len(live) + 1):
+            yield from take_unit(v)
+            if v == len(live):
+                break
+            yield from produce(g, range(v * nchunks, (v + 1) * nchunks))
+
+    def produce(g, its):
+        for it in its:
+            if it % groups != g:
+                continue
             ss, ks = it % SLAB, it // SLAB
             s, k = it % STAGES, it // STAGES
             yield ("wait", ("sfull", ss), ks & 1, ks + 1)
@@ -164,7 +218,7 @@ def simulate(units, nchunks, nprod, nepi, seed, async_bias, bad_reuse_parity=Fal
             yield ("arrive", ("sempty", ss), ks)
             yield ("arrive", ("ready", s), k)
 
-    roles = {"tma_slab": tma_slab(), "tma_rows": tma_rows(), "mma": mma()}
+    roles = {"scheduler": scheduler(), "tma_slab": tma_slab(), "tma_rows": tma_rows(), "mma": mma()}
     roles.update({f"epi{i}": epilogue() for i in range(nepi)})
     roles.update({f"prod{g}.{i}": producer(g) for g in range(groups) for i in range(nprod)})
     cur = {name: next(g, None) for name, g in roles.items()}
@@ -284,5 +338,20 @@ def test_access_checks_alone_catch_a_wrong_reuse_parity():
                      check_waits=False)
         except AssertionError as e:
             assert "overwritten" in str(e) or "deadlock" in str(e) or "phase" in str(e), str(e)
+            failures += 1
+    assert failures > 0
+
+
+def test_model_catches_a_missing_unit_slot_wait():
+    """A scheduler that refills a unit slot without waiting for every other
+    warp to have read it overwrites a unit some warp has not taken yet: the
+    access check reports it on some schedule (with more units than slots)."""
+    failures = 0
+    for trial in range(30):
+        try:
+            simulate([96, 16, 48] * 5, 1, nprod=1, nepi=1, seed=trial, async_bias=0.3, skip_slot_wait=True,
+                     check_waits=False, groups=2)
+        except AssertionError as e:
+            assert "unit slot" in str(e) or "deadlock" in str(e), str(e)
             failures += 1
     assert failures > 0
