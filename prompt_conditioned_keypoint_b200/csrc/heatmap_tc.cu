@@ -76,6 +76,7 @@ constexpr int kBBytes = 2 * kBSubBytes;          // 40 KB per stage, 1 KB aligne
 constexpr int kStoreReps = GKD_STORE_REPS;       // 16x256b repetitions per producer store (1, 2 or 4)
 static_assert(kStoreReps == 1 || kStoreReps == 2 || kStoreReps == 4, "producer store width");
 constexpr int kEpiCols = 16;
+
 constexpr int kDecCols = 8;                      // prompt rows per decode-mode block (len is a multiple of 8)                     // accumulator columns per epilogue group
 constexpr int kEpiStride = 40;                   // floats per (column, row) line of the epilogue tile
 constexpr int kEpiBufBytes = kEpiCols * kUnitRows * kEpiStride * 4;   // 10 KB
@@ -391,10 +392,16 @@ __device__ __forceinline__ void st_shared_f32(uint32_t addr, uint32_t v) {
 // quadrant base, column of the stage). Channel group r (0..3) of sub-chunk hs
 // holds channels 64 hs + 16 r + 4 cq .. +3, i.e. columns 8 r + 2 cq, +1 of the
 // sub-chunk: repetition r of the 16x256b.x4 store. fp32 slabs hold 32 channels
-// per 128-byte plane line, bf16 slabs 64.
-template <bool BF16>
-__device__ __forceinline__ void produce_stage(uint32_t sp, const uint32_t (&base)[4], uint32_t plane_bytes,
-                                              uint32_t f20, const Column4& cg, uint32_t acol) {
+// per 128-byte plane line, bf16 slabs 64. tap[k] is the shared address of tap k
+// in the stage's first plane (slab stage base + line + swizzled chunk); the
+// stage base is 1024-byte aligned, so flipping chunk bits 4-6 of the sum is
+// the same as flipping them in the in-slab offset. F5D: the planes are one box
+// of 20 lines each (pitch 2560 B, which shifts the swizzle row by 4 from plane
+// to plane) instead of separate 3 KB boxes.
+template <bool BF16, bool F5D>
+__device__ __forceinline__ void produce_stage(const uint32_t (&tap)[4], const Column4& cg, uint32_t acol) {
+  constexpr uint32_t plane_bytes = F5D ? kSlabLines * 128u : static_cast<uint32_t>(kPlaneSplit);
+  constexpr uint32_t f20 = F5D ? 1u : 0u;
   // kStoreReps repetitions of the 16x256b pattern per store: 4 groups per store
   // (one store per sub-chunk and half quadrant) or 2 (half the live registers)
 #pragma unroll
@@ -408,22 +415,22 @@ __device__ __forceinline__ void produce_stage(uint32_t sp, const uint32_t (&base
       if (!BF16) {
         const int plane = 2 * hs + (r >> 1);
         const uint32_t flip = ((static_cast<uint32_t>(r & 1) ^ (f20 & static_cast<uint32_t>(r >> 1))) << 6);
-        const uint32_t pb = sp + static_cast<uint32_t>(plane) * plane_bytes;
-        const float4 f00 = ld_shared_f4(pb + (base[0] ^ flip));
-        const float4 f01 = ld_shared_f4(pb + (base[1] ^ flip));
-        const float4 f10 = ld_shared_f4(pb + (base[2] ^ flip));
-        const float4 f11 = ld_shared_f4(pb + (base[3] ^ flip));
+        const uint32_t po = static_cast<uint32_t>(plane) * plane_bytes;
+        const float4 f00 = ld_shared_f4((tap[0] ^ flip) + po);
+        const float4 f01 = ld_shared_f4((tap[1] ^ flip) + po);
+        const float4 f10 = ld_shared_f4((tap[2] ^ flip) + po);
+        const float4 f11 = ld_shared_f4((tap[3] ^ flip) + po);
         lerp_column(make_float2(f00.x, f00.y), make_float2(f01.x, f01.y), make_float2(f10.x, f10.y),
                     make_float2(f11.x, f11.y), cg, o[0]);
         lerp_column(make_float2(f00.z, f00.w), make_float2(f01.z, f01.w), make_float2(f10.z, f10.w),
                     make_float2(f11.z, f11.w), cg, o[1]);
       } else {
         const uint32_t flip = (static_cast<uint32_t>(2 * r) ^ (f20 * 4u * static_cast<uint32_t>(hs & 1))) << 4;
-        const uint32_t pb = sp + static_cast<uint32_t>(hs) * plane_bytes;
-        const uint2 u00 = ld_shared_u2(pb + (base[0] ^ flip));
-        const uint2 u01 = ld_shared_u2(pb + (base[1] ^ flip));
-        const uint2 u10 = ld_shared_u2(pb + (base[2] ^ flip));
-        const uint2 u11 = ld_shared_u2(pb + (base[3] ^ flip));
+        const uint32_t po = static_cast<uint32_t>(hs) * plane_bytes;
+        const uint2 u00 = ld_shared_u2((tap[0] ^ flip) + po);
+        const uint2 u01 = ld_shared_u2((tap[1] ^ flip) + po);
+        const uint2 u10 = ld_shared_u2((tap[2] ^ flip) + po);
+        const uint2 u11 = ld_shared_u2((tap[3] ^ flip) + po);
         lerp_column(bf16lo_hi(u00.x), bf16lo_hi(u01.x), bf16lo_hi(u10.x), bf16lo_hi(u11.x), cg, o[0]);
         lerp_column(bf16lo_hi(u00.y), bf16lo_hi(u01.y), bf16lo_hi(u10.y), bf16lo_hi(u11.y), cg, o[1]);
       }
@@ -786,6 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
       }
       float* hb = a.heat + static_cast<long long>(b) * a.M * a.K * P;
       const int shift0 = ci.kmin0, shift1 = a.K + ci.kmin1 - ci.off1;
+
       const int ngroups = ci.n / kEpiCols;
       if (half >= ngroups) {   // no column group for this set: release the accumulator now
         tc_fence_before();
@@ -943,8 +951,6 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
     const int grp = (warp - kWarpProd0) / kProdGroupWarps;
     const int jx = lane >> 2, cq = lane & 3;            // column within the quadrant, 4-channel group
     const bool skip_first = (a.debug_flags & kDbgSkipProducerArrive) != 0;
-    const uint32_t plane_bytes = (a.feat_5d ? kSlabLines : kPlaneSplit / 128) * 128u;
-    const uint32_t f20 = a.feat_5d ? 1u : 0u;          // plane pitch of 20 lines shifts the swizzle row by 4
     uint32_t it = 0;
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
@@ -980,16 +986,23 @@ __global__ void __launch_bounds__(kThreads, 1) heatmap_tc_kernel(const __grid_co
         }
         tc_fence_after();
         if (lane == 0 && (warp - kWarpProd0) % kProdGroupWarps == 0) GKD_TR(6, s_it);
-        const uint32_t sp = smem_base + ss * kSlabBytes;
+        const uint32_t sp = smem_base + ss * kSlabBytes;   // 1024-byte aligned
         const uint32_t acol = tmem + kColA + st * 64 + (static_cast<uint32_t>(32 * q) << 16);
-        // opaque per stage: keeps the compiler from hoisting the 16 swizzled tap
-        // addresses of the stage out of the loop (registers it does not have)
+        uint32_t tap[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) asm volatile("" : "+r"(base[k]));
-        if (a.feat_bf16)
-          produce_stage<true>(sp, base, plane_bytes, f20, cg, acol);
-        else
-          produce_stage<false>(sp, base, plane_bytes, f20, cg, acol);
+        for (int k = 0; k < 4; ++k) {
+          tap[k] = sp + base[k];
+          // opaque per stage: keeps the compiler from hoisting the 16 swizzled tap
+          // addresses of the stage out of the loop (registers it does not have)
+          asm volatile("" : "+r"(tap[k]));
+        }
+        if (a.feat_bf16) {
+          if (a.feat_5d) produce_stage<true, true>(tap, cg, acol);
+          else produce_stage<true, false>(tap, cg, acol);
+        } else {
+          if (a.feat_5d) produce_stage<false, true>(tap, cg, acol);
+          else produce_stage<false, false>(tap, cg, acol);
+        }
         if (lane == 0 && (warp - kWarpProd0) % kProdGroupWarps == 0) GKD_TR(7, s_it);
         tmem_wait_st();
         tc_fence_before();
