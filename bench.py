@@ -354,6 +354,25 @@ def heatmap_smem_roofline(shape, mask, launch_s: float, sm_mhz: float | None) ->
             "roofline_us": m["bytes_per_launch"] / peak * 1e6}
 
 
+TF32_OVER_BF16 = 1.1 / 2.25        # nominal dense tf32 / bf16 tensor peaks of a B200
+
+
+def pool_roofline(flops: float, hbm: float, launch_s: float, peaks: dict) -> dict:
+    """Gaussian pooling as a tensor-core GEMM (tf32 operands): the bound is the
+    slower of its algorithmic FLOPs at the tf32 peak (the measured bf16 peak x
+    the nominal tf32/bf16 ratio) and its bytes at the measured HBM peak."""
+    peak_tf32 = peaks["bf16_tflops"] * TF32_OVER_BF16
+    t_tensor = flops / (peak_tf32 * 1e12)
+    t_hbm = hbm / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        ach = flops / launch_s / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": peak_tf32, "unit": "TFLOP/s", "frac": ach / peak_tf32,
+                "roofline_us": t_tensor * 1e6, "peak_note": "measured bf16 x nominal tf32/bf16"}
+    ach = hbm / launch_s / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+            "roofline_us": t_hbm * 1e6}
+
+
 def heatmap_roofline(shape, mask, launch_s: float, peaks: dict) -> dict:
     """Roofline of one gkd_heatmap launch of `launch_s` seconds: bf16 operands
     are bound by the slower of dense bf16 tensor time and HBM time; the fp32
@@ -512,8 +531,8 @@ def variant_timings(dev, stream, launches: int, peaks: dict, cfg: int = 2) -> di
                              "kernels": "contraction on the source grid (tcgen05) + upsample"}
     del head, G
     torch.cuda.empty_cache()
-    # pooling (FFMA-bound)
-    peak_alu = FFMA_TFLOPS
+    # pooling: a tf32 tensor-core GEMM per crop, bound by the slower of its
+    # FLOPs at the tf32 peak and its bytes at the HBM peak
     for pc in (1, 5):
         wp = S.make_config(pc)
         hs = HeadShape.of(wp)
@@ -526,10 +545,9 @@ def variant_timings(dev, stream, launches: int, peaks: dict, cfg: int = 2) -> di
         nk = float(np.asarray(wp.kmask).sum())
         pf = 2.0 * nk * hs.h * hs.w * hs.C
         pb = hs.B * hs.h * hs.w * hs.C * 4 + hs.B * hs.K * hs.C * 4
-        out[f"pool_w{pc}"] = {"bound": "alu", "achieved": pf / mean / 1e12, "peak": peak_alu, "unit": "TFLOP/s",
-                              "frac": pf / mean / 1e12 / peak_alu, "launch_us": 1e6 * mean,
-                              "launch_us_median": 1e6 * med, "algorithmic_flops_per_launch": pf,
-                              "algorithmic_bytes_per_launch": pb, "hbm_gbs": pb / mean / 1e9}
+        out[f"pool_w{pc}"] = dict(pool_roofline(pf, pb, mean, peaks), launch_us=1e6 * mean,
+                                  launch_us_median=1e6 * med, algorithmic_flops_per_launch=pf,
+                                  algorithmic_bytes_per_launch=pb, hbm_gbs=pb / mean / 1e9)
         del head
     torch.cuda.empty_cache()
     gk.gkd_check_device_error(stream)

@@ -101,7 +101,11 @@ typedef enum gkd_dtype {
  *            [K][C] contiguous (proto_batch_stride >= K * C; pass 2*K*C to
  *            write straight into modality 0 of a [B][2][K][C] row tensor).
  * Limits: 1 <= K <= 128, 1 <= h, w <= 256, B <= 65535, sigma_px > 0, stride_px > 0.
- * The sums are fp32; their order is fixed (it does not depend on scheduling).
+ * Computed as one tensor-core GEMM per crop (keypoints x pixels x channels):
+ * the weights and features are each carried as a pair of TF32 numbers
+ * (x = hi + lo), three products per term, fp32 accumulation in a fixed order
+ * (the result does not depend on scheduling); each term is within about
+ * 2^-21 of its fp32 product. Features must be finite.
  */
 GKD_API gkd_status gkd_pool_prototypes(const void* support, gkd_dtype sdt, int B, int h, int w, int C,
                                const float* kpts, const uint8_t* kmask, int K, float sigma_px,

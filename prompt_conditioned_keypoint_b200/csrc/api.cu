@@ -198,9 +198,15 @@ gkd_status gkd_pool_prototypes(const void* support, gkd_dtype sdt, int B, int h,
   GKD_TRY(check_same_device(kpts, "kpts", dev));
   GKD_TRY(check_same_device(kmask, "kmask", dev));
   GKD_TRY(check_same_device(proto, "proto", dev));
-  return launched(gkd::launch_pool(static_cast<const float*>(support), B, h, w, C, kpts, kmask, K, sigma_px,
-                                   stride_px, proto, proto_batch_stride, static_cast<cudaStream_t>(stream)),
-                  "pool");
+  DeviceState* ds = nullptr;
+  GKD_TRY(device_state(dev, &ds));
+  const char* why = "";
+  const cudaError_t e = gkd::launch_pool_tc(
+      static_cast<const float*>(support), B, h, w, C, kpts, kmask, K, sigma_px, stride_px, proto,
+      proto_batch_stride, ds->err_word, static_cast<unsigned long long>(g_wait_timeout_ms.load()) * 1000000ull,
+      ds->num_sms, static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess && why[0]) return fail(GKD_ERR_CUDA, "pool: %s", why);
+  return launched(e, "pool");
 }
 
 gkd_status gkd_norm_kernels(const float* rows, const uint8_t* mask, int Bk, int M, int K, int C, float eps,

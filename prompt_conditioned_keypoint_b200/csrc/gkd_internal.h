@@ -19,10 +19,6 @@ enum : unsigned {
   kDbgSkipProducerArrive = 1u << 0,   // upsample producers never signal their first stage
 };
 
-cudaError_t launch_pool(const float* support, int B, int h, int w, int C, const float* kpts,
-                        const uint8_t* kmask, int K, float sigma, float stride, float* proto,
-                        long long proto_batch_stride, cudaStream_t stream);
-
 cudaError_t launch_norm(const float* rows, const uint8_t* mask, long long nrows, int C, float eps,
                         bool out_bf16, void* out, cudaStream_t stream);
 
@@ -88,6 +84,25 @@ struct ContractArgs {
 
 cudaError_t launch_contract_first(ContractArgs& a, const void* feat, const void* kern, long long kern_batch_stride,
                                   float* heat, cudaStream_t stream, const char** why);
+
+// Gaussian prototype pooling on the tensor cores (pool_tc.cu).
+struct PoolTcArgs {
+  CUtensorMap tmap;                      // support features as {C, h*w, B} fp32, box {32, 32, 1}
+  const float* kpts;                     // [B][K][2]
+  const uint8_t* kmask;                  // [B][K]
+  float* proto;
+  long long proto_bs;
+  int h, w, C, K;
+  int N;                                 // channels per CTA (32..256, a multiple of 32)
+  float sigma, stride;
+  unsigned* err;
+  unsigned long long wait_limit_ns;
+};
+
+cudaError_t launch_pool_tc(const float* support, int B, int h, int w, int C, const float* kpts,
+                           const uint8_t* kmask, int K, float sigma, float stride, float* proto,
+                           long long proto_batch_stride, unsigned* err, unsigned long long wait_limit_ns,
+                           int num_sms, cudaStream_t stream, const char** why);
 
 // cuTensorMapEncodeTiled resolved through the runtime's driver entry point.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

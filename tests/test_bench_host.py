@@ -156,3 +156,12 @@ def test_heatmap_smem_model_arithmetic():
     assert r["bound"] == "smem" and abs(r["frac"] - m["bytes_per_launch"] / 1e-3 / peak) < 1e-12
     assert bench.heatmap_smem_roofline(HeadShape(B=1, h=24, w=24, C=256, K=80, M=1, kern_dtype="f32"),
                                        mask[:1, :1], 1e-3, None) is None
+
+
+def test_pool_roofline_bound():
+    """Pooling is bound by the slower of tf32 tensor time and HBM time."""
+    peaks = {"bf16_tflops": 2250.0, "hbm_gbs": 1000.0}
+    r = bench.pool_roofline(1.0e9, 1.0e9, 2e-3, peaks)            # HBM: 1 ms; tensor: ~0.9 us
+    assert r["bound"] == "hbm" and abs(r["frac"] - 0.5) < 1e-12 and abs(r["roofline_us"] - 1000.0) < 1e-9
+    r = bench.pool_roofline(1.1e15, 1.0, 2.0, peaks)              # tensor: 1 s at 1100 TFLOP/s
+    assert r["bound"] == "tensor" and abs(r["peak"] - 1100.0) < 1e-6 and abs(r["frac"] - 0.5) < 1e-9
