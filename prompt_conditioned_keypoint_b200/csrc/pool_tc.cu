@@ -21,7 +21,7 @@
 // One CTA per (crop, block of N <= 256 channels), 14 warps:
 //   warp 0      TMA: per stage of 32 pixels, the [32 px][N ch] fp32 feature tile
 //               (boxes of 32 pixels x 32 channels; pixels past h*w and channels
-//               past C read as zeros) into a 2-deep raw ring;
+//               past C read as zeros) into a 3-deep raw ring;
 //   warp 1      MMA: per stage, 4 K-steps x 3 products, into an N-column fp32
 //               accumulator; one commit frees the stage;
 //   warps 2-5   weights (one thread per keypoint = tensor-memory lane): the
@@ -30,7 +30,8 @@
 //               they also sum the keypoint's weights in pixel order and, at the
 //               end, scale and store the prototypes;
 //   warps 6-13  converters (one thread per channel): the stage's raw tile split
-//               hi/lo and transposed into two K-major, 128B-swizzled B tiles.
+//               hi/lo and transposed into two K-major, 128B-swizzled B tiles
+//               (2-deep, as are the A stages in tensor memory).
 // Every wait is bounded; a timeout sets the device error word and every role
 // drains what it has in flight.
 #include "gkd_internal.h"
