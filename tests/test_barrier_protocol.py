@@ -355,3 +355,31 @@ def test_model_catches_a_missing_unit_slot_wait():
             assert "unit slot" in str(e) or "deadlock" in str(e), str(e)
             failures += 1
     assert failures > 0
+
+
+def _epilogue_set_decisions(seed, agree):
+    """Four epilogue warps of a set wait on accfull with a bounded wait that
+    tests the phase first and, while it is incomplete, gives up once the abort
+    flag is set. The MMA's commit and another role's abort land at random times,
+    and the warps reach their wait at random times. A warp that arrives after
+    the commit succeeds; one that arrives before it succeeds only if the commit
+    comes before the abort. With `agree` the set takes one decision (the AND
+    over its warps, as bar.red.and gives); without it each warp acts alone."""
+    rnd = random.Random(seed)
+    commit_at, abort_at = rnd.randint(0, 9), rnd.randint(0, 9)
+    starts = [rnd.randint(0, 9) for _ in range(4)]
+    own = [t >= commit_at or commit_at <= abort_at for t in starts]
+    return [all(own)] * 4 if agree else own
+
+
+def test_epilogue_set_takes_one_decision_on_abort():
+    """The kernel's epilogue warps meet at named barriers after the accumulator
+    wait, so every warp of a set must take the same path when an abort lands as
+    the commit completes; the AND-reduced decision guarantees it, per-warp
+    decisions do not (on some schedule a warp would wait at a barrier the others
+    skipped)."""
+    split = 0
+    for seed in range(400):
+        assert len(set(_epilogue_set_decisions(seed, agree=True))) == 1
+        split += len(set(_epilogue_set_decisions(seed, agree=False))) > 1
+    assert split > 0
