@@ -16,7 +16,9 @@
 //                    x-lerps on the two source rows, then the y-lerp.
 //
 // 16x fewer multiply-adds than the graded path; the heatmap writes dominate, so
-// the pair is bound by HBM. One CTA per unit (no persistence): the GEMM is small.
+// the pair is bound by HBM. One CTA per unit (no persistence): the GEMM is small,
+// so each CTA takes half an SM (104 KB of shared memory, 256 tensor-memory
+// columns) and two CTAs overlap each other's load latency.
 // Every wait is bounded; on a timeout the CTA records it and drains.
 #include "gkd_internal.h"
 #include "ptx.cuh"
@@ -24,7 +26,7 @@
 namespace gkd {
 namespace cf {
 
-constexpr int kStages = 4;                          // ring of 64-channel stages
+constexpr int kStages = 2;                          // ring of 64-channel stages (two CTAs share an SM)
 constexpr int kChunk = 64;
 constexpr int kMaxN = 160;
 constexpr int kTile = 128;                          // source pixels per unit (TMEM lanes)
@@ -32,7 +34,7 @@ constexpr int kFeatBytes = kTile * 256;             // fp32: two 128-byte planes
 constexpr int kBBytes = kMaxN * 128;                // kernel rows of a stage, 64 bf16 channels each
 constexpr int kWarps = 6;                           // 0 TMA, 1 MMA, 2-5 convert + epilogue
 constexpr int kThreads = kWarps * 32;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 256;                 // accumulator (<= 160) + two 32-column A stages
 constexpr uint32_t kColA = kMaxN;                   // accumulator at 0, A stages at 160 + 32 s
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * (kFeatBytes + kBBytes) + 256;
 
@@ -83,7 +85,7 @@ __device__ __forceinline__ uint64_t make_bdesc(uint32_t smem_addr) {
          (2ull << 61);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) contract_kernel(const __grid_constant__ ContractArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) contract_kernel(const __grid_constant__ ContractArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* bring = smem + kStages * kFeatBytes;
@@ -277,8 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1) contract_kernel(const __grid_cons
 
 // heat[b,m,k] = Up(G[b,m,k]) for valid rows; one CTA per (crop, row): the row's
 // source-grid map is staged in shared memory once (read in place from global
-// memory when it does not fit, STAGED = false), then every thread writes 4
-// output pixels (one float4, streaming) per step.
+// memory when it does not fit, STAGED = false). A thread's work item is a band
+// of four output rows (Y = 4s+2 .. 4s+5, which all read source rows s and s+1,
+// clamped at the borders) by four consecutive output columns: it x-lerps the
+// four columns on the two source rows once and y-lerps them into the band's
+// rows, one float4 (streaming) per row. The arithmetic per pixel is that of
+// the plain rule: x-lerps on the two source rows, then the y-lerp.
 template <bool STAGED>
 __global__ void __launch_bounds__(256) upsample_kernel(const float* __restrict__ G, const uint8_t* __restrict__ mask,
                                                        long long mask_bs, int M, int K, int h, int w,
@@ -295,24 +301,37 @@ __global__ void __launch_bounds__(256) upsample_kernel(const float* __restrict__
     gs = gsm;
   }
   float* out = heat + (static_cast<long long>(b) * M * K + row) * static_cast<long long>(H) * W;
-  for (int q = threadIdx.x; q < H * W / 4; q += blockDim.x) {
-    const int Y = (4 * q) / W, X0 = (4 * q) % W;
-    const float sy = fmaxf((static_cast<float>(Y) + 0.5f) * 0.25f - 0.5f, 0.f);
-    const int i0 = static_cast<int>(sy), i1 = min(i0 + 1, h - 1);
-    const float ly = sy - static_cast<float>(i0);
+  const int nitems = (h + 1) * w;                      // bands x float4 columns
+  for (int it = threadIdx.x; it < nitems; it += blockDim.x) {
+    const int band = it / w, u = it - band * w;
+    const int Yb = 4 * band - 2;                        // the band's first output row (may be < 0)
+    // source rows of the band, from its first row inside the map
+    const int Yf = max(Yb, 0);
+    const float sy0 = fmaxf((static_cast<float>(Yf) + 0.5f) * 0.25f - 0.5f, 0.f);
+    const int i0 = static_cast<int>(sy0), i1 = min(i0 + 1, h - 1);
     const float* r0 = gs + i0 * w;
     const float* r1 = gs + i1 * w;
-    float v[4];
+    float t0[4], t1[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int X = X0 + e;
+      const int X = 4 * u + e;
       const float sx = fmaxf((static_cast<float>(X) + 0.5f) * 0.25f - 0.5f, 0.f);
       const int j0 = static_cast<int>(sx), j1 = min(j0 + 1, w - 1);
       const float lx = sx - static_cast<float>(j0);
-      const float t0 = fmaf(lx, r0[j1] - r0[j0], r0[j0]), t1 = fmaf(lx, r1[j1] - r1[j0], r1[j0]);
-      v[e] = fmaf(ly, t1 - t0, t0);
+      t0[e] = fmaf(lx, r0[j1] - r0[j0], r0[j0]);
+      t1[e] = fmaf(lx, r1[j1] - r1[j0], r1[j0]);
     }
-    __stcs(reinterpret_cast<float4*>(out) + q, make_float4(v[0], v[1], v[2], v[3]));
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int Y = Yb + t;
+      if (Y < 0 || Y >= H) continue;
+      const float sy = fmaxf((static_cast<float>(Y) + 0.5f) * 0.25f - 0.5f, 0.f);
+      const float ly = sy - static_cast<float>(i0);
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = fmaf(ly, t1[e] - t0[e], t0[e]);
+      __stcs(reinterpret_cast<float4*>(out + static_cast<long long>(Y) * W) + u, make_float4(v[0], v[1], v[2], v[3]));
+    }
   }
 }
 
