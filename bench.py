@@ -292,68 +292,6 @@ def heatmap_algorithmic(shape, mask) -> tuple[float, float]:
     return flops, hbm
 
 
-SMEM_BYTES_PER_CLK = 128          # shared-memory bandwidth of one SM (32 banks x 4 B per clock)
-
-
-def accumulator_columns(mask_row, K: int) -> int:
-    """Accumulator columns the tensor-core kernel gives one crop: the contiguous
-    valid segment of each modality, each rounded up to 8, the total to 16."""
-    m = np.asarray(mask_row).reshape(-1, K)
-    used = 0
-    for row in m:
-        idx = np.nonzero(row)[0]
-        if len(idx):
-            used += (int(idx[-1]) - int(idx[0]) + 1 + 7) // 8 * 8
-    return (used + 15) // 16 * 16
-
-
-def heatmap_smem_model(shape, mask) -> dict:
-    """Shared-memory bytes one launch of the tensor-core heatmap kernel moves, by
-    the kernel's design. Per 128-channel stage of a 128-pixel unit with n
-    accumulator columns: the feature slab's TMA write (2 x 10 source pixels x
-    128 channels), the producers' tap reads (each thread reads 4 taps x 32
-    channels for its 4 pixels: 128 px x 128 ch x 4 taps x elt / 4), the kernel
-    rows' TMA write and the MMA's read of them (n x 128 ch x 2 B each), and the
-    epilogue's transpose through the shared tile (write + read of n x 128 px x
-    4 B per unit, i.e. n x 128 B per stage)."""
-    nb = int(np.asarray(mask).shape[0])
-    ns = [accumulator_columns(np.asarray(mask)[b], shape.K) for b in range(nb)]
-    if shape.shared:
-        ns = ns * shape.B if nb == 1 else ns
-    elt = 2 if shape.feat_dtype == "bf16" else 4
-    nbands = (shape.H + 2 + 3) // 4
-    ncb = (shape.W + 31) // 32
-    stages_per_unit = (shape.C + 127) // 128
-    slab = 2 * 10 * 128 * elt
-    taps = 128 * 128 * 4 * elt // 4
-    total = 0.0
-    stages = 0
-    for n in ns:
-        if n == 0:
-            continue
-        per_stage = slab + taps + 2 * n * 128 * 2 + n * 128
-        units = nbands * ncb
-        total += units * stages_per_unit * per_stage
-        stages += units * stages_per_unit
-    return {"bytes_per_launch": total, "stages": stages,
-            "bytes_per_stage_mean": total / stages if stages else 0.0}
-
-
-def heatmap_smem_roofline(shape, mask, launch_s: float, sm_mhz: float | None) -> dict | None:
-    """The tensor-core heatmap kernel against the SMs' shared-memory bandwidth
-    (148 SMs x 128 B per clock), at the SM clock sampled during the run (else
-    the maximum, 1965 MHz)."""
-    if shape.kern_dtype != "bf16":
-        return None
-    m = heatmap_smem_model(shape, mask)
-    mhz = sm_mhz or 1965.0
-    peak = 148 * SMEM_BYTES_PER_CLK * mhz * 1e6
-    ach = m["bytes_per_launch"] / launch_s
-    return {"bound": "smem", "bytes_per_launch": m["bytes_per_launch"], "bytes_per_stage_mean": m["bytes_per_stage_mean"],
-            "achieved": ach / 1e9, "peak": peak / 1e9, "unit": "GB/s", "frac": ach / peak, "sm_mhz": mhz,
-            "roofline_us": m["bytes_per_launch"] / peak * 1e6}
-
-
 TF32_OVER_BF16 = 1.1 / 2.25        # nominal dense tf32 / bf16 tensor peaks of a B200
 
 
@@ -398,7 +336,7 @@ def heatmap_roofline(shape, mask, launch_s: float, peaks: dict) -> dict:
     return roof
 
 
-def per_workload_heatmaps(dev, stream, launches: int, peaks: dict, cfgs=(1, 2, 3, 4, 5), sm_mhz=None) -> dict:
+def per_workload_heatmaps(dev, stream, launches: int, peaks: dict, cfgs=(1, 2, 3, 4, 5)) -> dict:
     """gkd_heatmap alone on each workload at full size: `launches` timed launches
     (CUDA events around each, on the launching stream) after 3 warm-up ones.
     Workload 1 fits in L2, so a 256 MB buffer is written between its launches
@@ -433,7 +371,6 @@ def per_workload_heatmaps(dev, stream, launches: int, peaks: dict, cfgs=(1, 2, 3
         gk.gkd_check_device_error(stream)
         ts = [a.elapsed_time(b) / 1e3 for a, b in evs]
         roof = heatmap_roofline(shape, wl.mask, sum(ts) / len(ts), peaks)
-        roof["smem"] = heatmap_smem_roofline(shape, wl.mask, sum(ts) / len(ts), sm_mhz)
         roof.update({"launch_us_median": 1e6 * statistics.median(ts), "launch_us_min": 1e6 * min(ts),
                      "launches": len(ts), "workload": S.CONFIG_NAMES[cfg],
                      "crops_per_s_heatmap": shape.B / (sum(ts) / len(ts)),
@@ -634,7 +571,6 @@ def main(argv=None):
                            l2="inputs larger than L2 (features + heatmaps per step exceed 126 MB)"),
             "heatmap_gflops": flops / hm_s / 1e9, "roofline": roof,
             "gpu_launches": args.steps * shape.launches_per_step(), "clocks": clocks.summary()}
-    roof["smem"] = heatmap_smem_roofline(shape, wl.mask, hm_s, line["clocks"].get("sm_mhz"))
 
     # end to end through the public API: pinned host inputs in, decoded keypoints out
     if not args.no_e2e:
@@ -658,8 +594,7 @@ def main(argv=None):
     gk.gkd_check_device_error(stream)
 
     if world == 1 and not args.no_per_workload:
-        line["per_workload"] = per_workload_heatmaps(dev, stream, args.per_workload_launches, peaks,
-                                                     sm_mhz=line["clocks"].get("sm_mhz"))
+        line["per_workload"] = per_workload_heatmaps(dev, stream, args.per_workload_launches, peaks)
     if world == 1 and not args.no_variants:
         line["variants"] = variant_timings(dev, stream, args.per_workload_launches, peaks)
 

@@ -1,4 +1,4 @@
-"""ctypes binding of libgkd (include/gkd.h), entry point for entry point.
+"""ctypes binding of libgkd (include/gkd.h), one Python function per C entry point.
 
 Argument marshalling only: every function here turns tensors into device
 pointers and sizes, calls the C ABI, and raises GkdError on a non-OK status.

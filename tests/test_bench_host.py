@@ -130,34 +130,6 @@ def test_heatmap_roofline_arithmetic():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and abs(r["achieved"] - hbm / 1e9) < 1e-9
 
 
-def test_heatmap_smem_model_arithmetic():
-    """Shared-memory bytes of a tensor-core heatmap launch by the kernel's design,
-    counted by hand for one crop: accumulator columns are each modality's valid
-    segment rounded up to 8, the total to 16; a 96x96 output has 25 bands x 3
-    column blocks of units; C = 256 gives 2 stages per unit."""
-    import numpy as np
-
-    from prompt_conditioned_keypoint_b200.head import HeadShape
-    mask = np.zeros((2, 2, 80), np.uint8)
-    mask[0, 0, 3:12] = 1         # segment of 9 -> 16 columns
-    mask[0, 1, 40] = 1           # one row -> 8 columns; 24 -> 32 in all
-    assert bench.accumulator_columns(mask[0], 80) == 32
-    assert bench.accumulator_columns(mask[1], 80) == 0
-    shape = HeadShape(B=2, h=24, w=24, C=256, K=80, M=2, feat_dtype="f32", kern_dtype="bf16")
-    m = bench.heatmap_smem_model(shape, mask)
-    per_stage = 2 * 10 * 128 * 4 + 128 * 128 * 4 * 4 // 4 + 2 * 32 * 256 + 32 * 128
-    assert m["stages"] == 25 * 3 * 2                # the empty crop does no work
-    assert m["bytes_per_launch"] == 25 * 3 * 2 * per_stage
-    bf = HeadShape(B=2, h=24, w=24, C=256, K=80, M=2, feat_dtype="bf16", kern_dtype="bf16")
-    per_stage_bf = 2 * 10 * 128 * 2 + 128 * 128 * 4 * 2 // 4 + 2 * 32 * 256 + 32 * 128
-    assert bench.heatmap_smem_model(bf, mask)["bytes_per_launch"] == 25 * 3 * 2 * per_stage_bf
-    r = bench.heatmap_smem_roofline(shape, mask, 1e-3, 1000.0)
-    peak = 148 * 128 * 1000e6
-    assert r["bound"] == "smem" and abs(r["frac"] - m["bytes_per_launch"] / 1e-3 / peak) < 1e-12
-    assert bench.heatmap_smem_roofline(HeadShape(B=1, h=24, w=24, C=256, K=80, M=1, kern_dtype="f32"),
-                                       mask[:1, :1], 1e-3, None) is None
-
-
 def test_pool_roofline_bound():
     """Pooling is bound by the slower of tf32 tensor time and HBM time."""
     peaks = {"bf16_tflops": 2250.0, "hbm_gbs": 1000.0}
