@@ -310,8 +310,10 @@ gkd_status enqueue_heatmap_decode(int dev, const void* feat, gkd_dtype fdt, int 
   cudaError_t e = cudaMemsetAsync(keys, 0, sizeof(unsigned long long) * static_cast<size_t>(B) * K, st);
   if (e != cudaSuccess) return fail(GKD_ERR_CUDA, "scratch clear failed: %s", cudaGetErrorString(e));
   if (kdt == GKD_F32) {
+    DeviceState* ds = nullptr;
+    GKD_TRY(device_state(dev, &ds));
     e = gkd::launch_heatmap_f32(static_cast<const float*>(feat), B, h, w, C, static_cast<const float*>(kern),
-                                kern_batch_stride, mask, mask_batch_stride, M, K, nullptr, keys, st);
+                                kern_batch_stride, mask, mask_batch_stride, M, K, nullptr, keys, ds->num_sms, st);
     if (e != cudaSuccess) return fail(GKD_ERR_CUDA, "heatmap decode (fp32) launch failed: %s", cudaGetErrorString(e));
   } else {
     DeviceState* ds = nullptr;
@@ -345,13 +347,13 @@ gkd_status gkd_heatmap(const void* feat, gkd_dtype fdt, int B, int h, int w, int
   GKD_TRY(check_same_device(mask, "mask", dev));
   GKD_TRY(check_same_device(heat, "heat", dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DeviceState* ds = nullptr;
+  GKD_TRY(device_state(dev, &ds));
   if (kdt == GKD_F32)
     return launched(gkd::launch_heatmap_f32(static_cast<const float*>(feat), B, h, w, C,
                                             static_cast<const float*>(kern), kern_batch_stride, mask,
-                                            mask_batch_stride, M, K, heat, nullptr, st),
+                                            mask_batch_stride, M, K, heat, nullptr, ds->num_sms, st),
                     "heatmap (fp32)");
-  DeviceState* ds = nullptr;
-  GKD_TRY(device_state(dev, &ds));
   gkd::HeatmapTcArgs a = tc_args(ds, fdt, B, h, w, C, kern_batch_stride, mask, mask_batch_stride, M, K);
   a.heat = heat;
   const char* why = "";

@@ -52,22 +52,39 @@ struct Seg {
   int kmin[2], len[2], off1, n;
 };
 
-__device__ __forceinline__ Seg segments(const ContractArgs& a, const uint8_t* mb) {
+// Warp-cooperative (every lane gets the result): the valid-row segment of each
+// modality. Lane l reads mask bytes 8l .. 8l+7 of the crop's [M][K] mask (M K <=
+// 256), so the whole mask costs one memory latency.
+__device__ __forceinline__ Seg segments(const ContractArgs& a, const uint8_t* mb, int lane) {
   Seg g{};
+  const int total = a.M * a.K;
+  uint32_t lb = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int p = 8 * lane + i;
+    if (p < total && mb[p] != 0) lb |= 1u << i;
+  }
   int off = 0;
+#pragma unroll
   for (int m = 0; m < 2; ++m) {
     g.kmin[m] = 0;
     g.len[m] = 0;
-    if (m >= a.M) continue;
-    int first = -1, last = -1;
-    for (int k = 0; k < a.K; ++k)
-      if (mb[m * a.K + k]) {
-        if (first < 0) first = k;
-        last = k;
+    if (m < a.M) {
+      int first = a.K, last = -1;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int k = 8 * lane + i - m * a.K;
+        if (((lb >> i) & 1u) && k >= 0 && k < a.K) {
+          first = min(first, k);
+          last = max(last, k);
+        }
       }
-    if (last >= 0) {
-      g.kmin[m] = first;
-      g.len[m] = (last - first + 1 + 7) & ~7;
+      first = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<unsigned>(first)));
+      last = __reduce_max_sync(0xffffffffu, last);
+      if (last >= 0) {
+        g.kmin[m] = first;
+        g.len[m] = (last - first + 1 + 7) & ~7;
+      }
     }
     if (m == 0) g.off1 = g.len[0];
     off += g.len[m];
@@ -96,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 2) contract_kernel(const __grid_cons
   const int b = blockIdx.x / ntiles, tile = blockIdx.x % ntiles;
   const int px0 = tile * kTile;
   const uint8_t* mb = a.mask + static_cast<long long>(b) * a.mask_batch_stride;
-  const Seg sg = segments(a, mb);
+  const Seg sg = segments(a, mb, threadIdx.x & 31);
   if (sg.n == 0) return;                              // uniform: no valid row in this crop
   const int nst = (a.C + kChunk - 1) / kChunk;
   const uint64_t lim = a.wait_limit_ns;

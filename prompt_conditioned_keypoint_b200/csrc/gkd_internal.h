@@ -38,7 +38,8 @@ cudaError_t launch_fuse_decode(const float* heat, const uint8_t* mask, long long
 // keys non-null: decode mode (no heatmap; one peak key per (crop, row) merged into keys)
 cudaError_t launch_heatmap_f32(const float* feat, int B, int h, int w, int C, const float* kern,
                                long long kern_batch_stride, const uint8_t* mask, long long mask_batch_stride,
-                               int M, int K, float* heat, unsigned long long* keys, cudaStream_t stream);
+                               int M, int K, float* heat, unsigned long long* keys, int num_sms,
+                               cudaStream_t stream);
 
 // Turns peak keys [B][K] into idx / xy / score / valid (decode fused into the heatmap kernels).
 cudaError_t launch_finalize_keys(const unsigned long long* keys, const uint8_t* mask, long long mask_batch_stride,
