@@ -10,13 +10,15 @@
 // 32-channel chunks, one per quarter. Per round the CTA copies, with cp.async
 // into a double buffer, each quarter's chunk of the tile's source patch (the 3
 // source rows x 10 source columns every pixel of the tile reads) and of its
-// rows; the copies of round r + 1 are in flight while round r computes. A
+// rows; the copies of round r + 1 are in flight while round r computes (a
+// deeper ring measured no faster on one crop and slower on large batches). A
 // thread owns one pixel: it forms the pixel's upsampled slice of its quarter's
 // chunk from the patch (4 taps, dyadic weights) and contracts it against the
 // chunk's rows. The four partial sums of a pixel are added in quarter order
 // through shared memory at the end (a fixed order: the result does not depend
 // on scheduling). ROWS is 32, or 16 when the batch has too few tiles to fill
-// the SMs twice (a single crop: twice the CTAs, each upsampling again).
+// the SMs twice (a single crop: twice the CTAs, each upsampling again); a
+// crop's rows are split evenly over the groups it needs.
 //
 // Decode mode (`keys` non-null): a group holds ROWS/2 prompt rows with both
 // modality slots side by side, so each thread fuses its pixel's two heatmap
@@ -42,7 +44,7 @@ struct F32Buf {                                    // one round: every quarter's
 };
 
 template <int ROWS>
-constexpr size_t f32_smem_bytes() {
+constexpr size_t f32_smem_bytes() {   // the double buffer, or the partial sums that reuse it if larger
   return 2 * sizeof(F32Buf<ROWS>) > sizeof(float) * (kF32Quarters - 1) * ROWS * kF32Pix
              ? 2 * sizeof(F32Buf<ROWS>)
              : sizeof(float) * (kF32Quarters - 1) * ROWS * kF32Pix;
@@ -120,9 +122,15 @@ __global__ void __launch_bounds__(kF32Threads) heatmap_f32_kernel(
     if (lane == 0) s_nrows = n;
   }
   __syncthreads();
-  const int r0 = rg * ROWS;
-  if (r0 >= s_nrows) return;
-  const int nr = min(ROWS, s_nrows - r0);
+  // the crop's rows split evenly over as many groups of at most ROWS as it needs
+  // (17 rows: 9 + 8, not 16 + 1); decode mode keeps the slot pairs together
+  const int nrows = s_nrows;
+  const int ngroups = (nrows + ROWS - 1) / ROWS;
+  if (rg >= ngroups) return;
+  const int per = decode ? 2 * ((nrows / 2 + ngroups - 1) / ngroups) : (nrows + ngroups - 1) / ngroups;
+  const int r0 = rg * per;
+  if (r0 >= nrows) return;
+  const int nr = min(per, nrows - r0);
 
   const int px = threadIdx.x % kF32Pix, qc = threadIdx.x / kF32Pix;   // pixel, channel quarter
   const int Y = 4 * band + (px >> 5);
