@@ -267,17 +267,32 @@ __global__ void __launch_bounds__(kThreads, 2) contract_kernel(const __grid_cons
     if (__all_sync(0xffffffffu, okw)) {
       tc_fence_after();
       const bool pix_ok = px0 + r < hw;
+      // valid accumulator columns as bits (bit c of word g: column 32 g + c), one
+      // mask byte per lane and word, so the loop below reads no mask
+      uint32_t colw[5];
+#pragma unroll
+      for (int g = 0; g < 5; ++g) {
+        const int n = 32 * g + lane;
+        const int m = n < sg.off1 ? 0 : 1;
+        const int k = (m ? sg.kmin[1] : sg.kmin[0]) + n - (m ? sg.off1 : 0);
+        const bool v = n < sg.len[0] + sg.len[1] && k < a.K && mb[m * a.K + k] != 0;
+        colw[g] = __ballot_sync(0xffffffffu, v);
+      }
+      float* gcrop = a.G + static_cast<long long>(b) * a.M * a.K * hw + px0 + r;
       for (int n0 = 0; n0 < sg.n; n0 += 16) {
         uint32_t vv[16];
         tmem_ld_32x32b_x16(tmem + lane_off + n0, vv);
         tmem_wait_ld();
+        const int g = n0 >> 5;   // select without indexing (keeps colw in registers)
+        const uint32_t word = g == 0 ? colw[0] : g == 1 ? colw[1] : g == 2 ? colw[2] : g == 3 ? colw[3] : colw[4];
+        const uint32_t bits = (word >> (n0 & 31)) & 0xFFFFu;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int n = n0 + c;
           const int m = n < sg.off1 ? 0 : 1;
-          const int k = sg.kmin[m] + n - (m ? sg.off1 : 0);
-          if (n < sg.len[0] + sg.len[1] && k < a.K && mb[m * a.K + k] && pix_ok)
-            a.G[((static_cast<long long>(b) * a.M + m) * a.K + k) * hw + px0 + r] = __uint_as_float(vv[c]);
+          const int k = (m ? sg.kmin[1] : sg.kmin[0]) + n - (m ? sg.off1 : 0);
+          if (((bits >> c) & 1u) && pix_ok)
+            gcrop[(static_cast<long long>(m) * a.K + k) * hw] = __uint_as_float(vv[c]);
         }
       }
     } else if (lane == 0) {
