@@ -6,8 +6,9 @@
 //   contract_kernel  G[b,m,k,i,j] = sum_c khat[b,m,k,c] * bf16(F[b,i,j,c]) on the
 //                    h x w source grid: a tcgen05 GEMM per (crop, tile of 128
 //                    source pixels), M = pixels, N = the crop's valid rows, K = C.
-//                    Four warps turn each TMA-loaded 64-channel slab into the
-//                    bf16 A operand in tensor memory (one pixel per lane: fp32
+//                    Two groups of four warps take the 64-channel stages in
+//                    turn and turn each TMA-loaded slab into the bf16 A
+//                    operand in tensor memory (one pixel per lane: fp32
 //                    features rounded to nearest even, bf16 features copied);
 //                    TMA brings the kernel rows as the B operand; the fp32
 //                    accumulator is written to G, one row of the crop at a time.
@@ -32,7 +33,9 @@ constexpr int kMaxN = 160;
 constexpr int kTile = 128;                          // source pixels per unit (TMEM lanes)
 constexpr int kFeatBytes = kTile * 256;             // fp32: two 128-byte planes per pixel (bf16 uses one)
 constexpr int kBBytes = kMaxN * 128;                // kernel rows of a stage, 64 bf16 channels each
-constexpr int kWarps = 6;                           // 0 TMA, 1 MMA, 2-5 convert + epilogue
+constexpr int kWarps = 10;                          // 0 TMA, 1 MMA, 2-9 convert + epilogue (two groups of four)
+constexpr int kConvGroups = 2;                      // group g converts the stages s with s % 2 == g
+static_assert(kConvGroups == kStages, "a converter group owns one ring slot");
 constexpr int kThreads = kWarps * 32;
 constexpr uint32_t kTmemCols = 256;                 // accumulator (<= 160) + two 32-column A stages
 constexpr uint32_t kColA = kMaxN;                   // accumulator at 0, A stages at 160 + 32 s
@@ -214,10 +217,13 @@ __global__ void __launch_bounds__(kThreads, 2) contract_kernel(const __grid_cons
   } else {
     // ------------------------------------------------------------ convert, then epilogue
     const int q = warp & 3;                           // lane quadrant
+    const int grp = (warp - 2) >> 2;                  // converter group: stages grp, grp + 2, ...
     const int r = 32 * q + lane;                      // tile pixel of this thread
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
     bool ok = true;
-    for (uint32_t it = 0; it < static_cast<uint32_t>(nst); ++it) {
+    // the two groups alternate stages, so one group's TMEM-store wait overlaps
+    // the other group's conversion
+    for (uint32_t it = grp; it < static_cast<uint32_t>(nst); it += kConvGroups) {
       const uint32_t s = it % kStages, ph = (it / kStages) & 1;
       const bool okw = mbar_wait_bounded(&ctl->full[s], ph, lim, abortp);
       if (!__all_sync(0xffffffffu, okw)) {
@@ -279,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 2) contract_kernel(const __grid_cons
         colw[g] = __ballot_sync(0xffffffffu, v);
       }
       float* gcrop = a.G + static_cast<long long>(b) * a.M * a.K * hw + px0 + r;
-      for (int n0 = 0; n0 < sg.n; n0 += 16) {
+      for (int n0 = 16 * grp; n0 < sg.n; n0 += 16 * kConvGroups) {   // the groups take alternate 16-column chunks
         uint32_t vv[16];
         tmem_ld_32x32b_x16(tmem + lane_off + n0, vv);
         tmem_wait_ld();
