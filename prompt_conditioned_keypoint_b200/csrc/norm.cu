@@ -8,6 +8,29 @@
 
 namespace gkd {
 
+constexpr int kNormRegQ = 10;   // float4 per lane held in registers: rows of up to 1280 channels
+
+template <bool OUT_BF16>
+__device__ __forceinline__ void store_norm(void* out, long long row, int C, int i, const float4& v, float d,
+                                           bool valid) {
+  if (OUT_BF16) {
+    uint2 o = make_uint2(0u, 0u);
+    if (valid) {
+      o.x = pack_bf16x2(__fdiv_rn(v.x, d), __fdiv_rn(v.y, d));
+      o.y = pack_bf16x2(__fdiv_rn(v.z, d), __fdiv_rn(v.w, d));
+    }
+    reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + row * C)[i] = o;
+  } else {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (valid) o = make_float4(__fdiv_rn(v.x, d), __fdiv_rn(v.y, d), __fdiv_rn(v.z, d), __fdiv_rn(v.w, d));
+    reinterpret_cast<float4*>(static_cast<float*>(out) + row * C)[i] = o;
+  }
+}
+
+// One warp per row. Rows of up to 1280 channels are read once: every lane
+// issues all of its 128-bit loads before the first use, keeps them in
+// registers for the division pass, and sums its squares in channel order
+// (lane, lane + 32, ...), as the streaming loop for longer rows does.
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(256) norm_rows_kernel(const float* __restrict__ rows,
                                                         const uint8_t* __restrict__ mask, long long nrows,
@@ -18,40 +41,47 @@ __global__ void __launch_bounds__(256) norm_rows_kernel(const float* __restrict_
   const float4* src = reinterpret_cast<const float4*>(rows + row * C);
   const int nq = C >> 2;
   const bool valid = mask[row] != 0;
+  const bool in_regs = nq <= 32 * kNormRegQ;
+  float4 reg[kNormRegQ];
   float ss = 0.f;
   if (valid) {
-    for (int i = lane; i < nq; i += 32) {
-      const float4 v = __ldg(src + i);
-      ss = fmaf(v.x, v.x, ss);
-      ss = fmaf(v.y, v.y, ss);
-      ss = fmaf(v.z, v.z, ss);
-      ss = fmaf(v.w, v.w, ss);
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < kNormRegQ; ++j) {
+        const int i = lane + 32 * j;
+        reg[j] = i < nq ? __ldg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < kNormRegQ; ++j) {
+        if (lane + 32 * j < nq) {
+          ss = fmaf(reg[j].x, reg[j].x, ss);
+          ss = fmaf(reg[j].y, reg[j].y, ss);
+          ss = fmaf(reg[j].z, reg[j].z, ss);
+          ss = fmaf(reg[j].w, reg[j].w, ss);
+        }
+      }
+    } else {
+      for (int i = lane; i < nq; i += 32) {
+        const float4 v = __ldg(src + i);
+        ss = fmaf(v.x, v.x, ss);
+        ss = fmaf(v.y, v.y, ss);
+        ss = fmaf(v.z, v.z, ss);
+        ss = fmaf(v.w, v.w, ss);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   }
   const float d = fmaxf(__fsqrt_rn(ss), eps);
-  if (OUT_BF16) {
-    uint2* dst = reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + row * C);
-    for (int i = lane; i < nq; i += 32) {
-      uint2 o = make_uint2(0u, 0u);
-      if (valid) {
-        const float4 v = __ldg(src + i);
-        o.x = pack_bf16x2(__fdiv_rn(v.x, d), __fdiv_rn(v.y, d));
-        o.y = pack_bf16x2(__fdiv_rn(v.z, d), __fdiv_rn(v.w, d));
-      }
-      dst[i] = o;
+  if (in_regs) {
+#pragma unroll
+    for (int j = 0; j < kNormRegQ; ++j) {
+      const int i = lane + 32 * j;
+      if (i < nq) store_norm<OUT_BF16>(out, row, C, i, reg[j], d, valid);
     }
   } else {
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row * C);
-    for (int i = lane; i < nq; i += 32) {
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (valid) {
-        const float4 v = __ldg(src + i);
-        o = make_float4(__fdiv_rn(v.x, d), __fdiv_rn(v.y, d), __fdiv_rn(v.z, d), __fdiv_rn(v.w, d));
-      }
-      dst[i] = o;
-    }
+    for (int i = lane; i < nq; i += 32)
+      store_norm<OUT_BF16>(out, row, C, i, valid ? __ldg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f), d, valid);
   }
 }
 
