@@ -504,7 +504,7 @@ def main(argv=None):
 
     import torch
     from prompt_conditioned_keypoint_b200 import binding as gk
-    from prompt_conditioned_keypoint_b200.head import GkdHead, HeadShape
+    from prompt_conditioned_keypoint_b200.head import GkdHead, HeadPipeline, HeadShape
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -572,25 +572,40 @@ def main(argv=None):
             "heatmap_gflops": flops / hm_s / 1e9, "roofline": roof,
             "gpu_launches": args.steps * shape.launches_per_step(), "clocks": clocks.summary()}
 
-    # end to end through the public API: pinned host inputs in, decoded keypoints out
+    # end to end through the public API: pinned host inputs in, decoded keypoints
+    # out, every step. Headline: HeadPipeline (two heads; the copy of step i + 1
+    # overlaps the head on step i). Also reported: one head, one step after the other.
     if not args.no_e2e:
+        def timed_e2e(run_steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            run_steps(e0)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier()
+            return max_over_ranks(e0.elapsed_time(e1) / 1e3, pg, dev)
+
         outh = None
         for _ in range(3):
             outh = head.run_host(host, outh, stream)
-        stream.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
-        torch.cuda.synchronize(dev)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            outh = head.run_host(host, outh, stream)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        te = max_over_ranks(e0.elapsed_time(e1) / 1e3, pg, dev)
-        line["e2e"] = {"value": job_throughput(world, shape.B, args.e2e_steps, te), "unit": UNIT,
+
+        def sequential(_e0):
+            for _ in range(args.e2e_steps):
+                head.run_host(host, outh, stream)
+
+        t_seq = timed_e2e(sequential)
+        pipe = HeadPipeline(shape, dev)
+        warm = pipe.run([host] * 3, None, stream)
+        outs = [warm[-1]] * args.e2e_steps
+        t_pipe = timed_e2e(lambda e0: pipe.run([host] * args.e2e_steps, outs, stream, start_event=e0))
+        line["e2e"] = {"value": job_throughput(world, shape.B, args.e2e_steps, t_pipe), "unit": UNIT,
                        "h2d_bytes_per_step": head.host_input_bytes(host), "d2h_bytes_per_step": head.output_bytes(),
-                       "steps": args.e2e_steps}
+                       "steps": args.e2e_steps, "api": "HeadPipeline.run (copies of step i + 1 overlap the head on step i)",
+                       "sequential": {"value": job_throughput(world, shape.B, args.e2e_steps, t_seq), "unit": UNIT,
+                                      "api": "GkdHead.run_host, one step after the other"}}
+        del pipe, warm, outs
     gk.gkd_check_device_error(stream)
 
     if world == 1 and not args.no_per_workload:

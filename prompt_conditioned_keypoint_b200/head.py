@@ -234,3 +234,43 @@ class GkdHead:
         rows = m.reshape(m.shape[0], -1).sum(axis=1).astype(np.float64)
         total_rows = rows[0] * s.B if s.shared else rows.sum()
         return 2.0 * total_rows * s.C * s.H * s.W
+
+
+class HeadPipeline:
+    """Two heads of one shape for a stream of batches: the host-to-device copy
+    of batch i + 1 runs on a copy stream while the head works on batch i on the
+    compute stream, so each batch costs the longer of the two instead of their
+    sum. Batch i's decoded outputs are copied to host on the compute stream
+    right after its head."""
+
+    def __init__(self, shape: HeadShape, device, **head_kw):
+        self.device = torch.device(device)
+        self.heads = [GkdHead(shape, self.device, **head_kw), GkdHead(shape, self.device, **head_kw)]
+        self.copy_stream = torch.cuda.Stream(self.device)
+        self._consumed = [None, None]   # per head: event after the last head that read its inputs
+
+    def run(self, hosts, outs=None, stream=None, start_event=None) -> list:
+        """Enqueue every batch of `hosts` (dicts as `GkdHead.host_inputs` gives,
+        pinned) and return one host output dict per batch (`outs[i]` when
+        given; a dict passed twice is overwritten by the later batch).
+        `start_event`, if given, is waited on before the first copy. Keep the
+        host tensors alive and synchronise `stream` before reading the outputs."""
+        st = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if start_event is not None:
+            self.copy_stream.wait_event(start_event)
+        res = []
+        for i, host in enumerate(hosts):
+            j = i & 1
+            head = self.heads[j]
+            if self._consumed[j] is not None:          # the head's previous batch has been read
+                self.copy_stream.wait_event(self._consumed[j])
+            head.upload(host, self.copy_stream)
+            landed = torch.cuda.Event()
+            landed.record(self.copy_stream)
+            st.wait_event(landed)
+            head.forward(st)
+            consumed = torch.cuda.Event()
+            consumed.record(st)
+            self._consumed[j] = consumed
+            res.append(head.outputs_to_host(outs[i] if outs is not None else None, st))
+        return res
