@@ -37,3 +37,26 @@ def test_pipeline_matches_one_batch_at_a_time(feat_dtype):
     gk.gkd_check_device_error()
     for i, g in zip(order, got):
         _same(ref[i], g)
+
+
+def test_pipeline_pooled_fp32_workload():
+    """Workload 1's shape (pooled prototypes, fp32 kernel rows): every input the
+    pipeline uploads (support map, keypoints, masks, features) goes through it."""
+    wl = S.make_config(1)
+    shape = HeadShape.of(wl)
+    single = GkdHead(shape, dev())
+    a = single.host_inputs(wl, pin=True)
+    b = {k: torch.empty_like(v, pin_memory=True).copy_(v) for k, v in a.items()}
+    b["feat"].neg_()                              # a second batch with other peaks
+    b["support"].mul_(0.5)
+    st = torch.cuda.current_stream(dev())
+    ref = []
+    for h in (a, b):
+        ref.append(single.run_host(h, None, st))
+        st.synchronize()
+    pipe = HeadPipeline(shape, dev())
+    got = pipe.run([a, b, b, a], None, st)
+    st.synchronize()
+    gk.gkd_check_device_error()
+    for i, g in zip((0, 1, 1, 0), got):
+        _same(ref[i], g)
