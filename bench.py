@@ -407,8 +407,11 @@ def variant_timings(dev, stream, launches: int, peaks: dict, cfg: int = 2) -> di
       heatmap launch against its tensor roofline (flops on the fused rows);
     - contract_first: contraction on the source grid + upsample, against HBM
       (features + kernel rows + G written and read + heatmaps written);
-    - pool: the pooling kernel on the pooled workloads (1, 5), against the FFMA
-      rate (its FLOPs exceed its bytes: 2 K h w C per crop over the full grid)."""
+    - pool: the pooling kernel on the pooled workloads (1, 5), against the
+      slower of its tf32 tensor time and its HBM time;
+    - preprocess / roi_to_image: the steps either side of the head, one box per
+      crop of the workload (canvases written against HBM; the point map is a
+      launch-latency-scale kernel)."""
     import torch
     from prompt_conditioned_keypoint_b200 import binding as gk
     from prompt_conditioned_keypoint_b200 import synthetic as S
@@ -487,6 +490,30 @@ def variant_timings(dev, stream, launches: int, peaks: dict, cfg: int = 2) -> di
                                   algorithmic_bytes_per_launch=pb, hbm_gbs=pb / mean / 1e9)
         del head
     torch.cuda.empty_cache()
+    # the steps either side of the head: one 1080p frame, one box per crop of the
+    # workload, 384x384 canvases; then the decoded points back to image pixels
+    Hi, Wi, canvas = 1080, 1920, 384
+    img, boxes = S.random_image_and_boxes(7, Hi, Wi, shape.B)
+    img_d = torch.from_numpy(img).to(dev)
+    boxes_d = torch.from_numpy(boxes).to(dev)
+    canv = torch.empty((shape.B, 3, canvas, canvas), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        med, mean, mn = _time_launches(lambda: gk.gkd_preprocess(img_d, Hi, Wi, boxes_d, shape.B, canvas, canv, stream),
+                                       stream, launches)
+    pb = canv.numel() * 4 + img.nbytes          # canvases written once, the frame read once
+    ach = pb / mean / 1e9
+    out["preprocess"] = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"], "launch_us": 1e6 * mean, "launch_us_median": 1e6 * med,
+                         "algorithmic_bytes_per_launch": pb,
+                         "workload": f"{shape.B} boxes of a {Wi}x{Hi} RGB frame -> {canvas}x{canvas} fp32 canvases"}
+    xy = torch.zeros((shape.B, shape.K, 2), dtype=torch.float32, device=dev)
+    pts = torch.empty_like(xy)
+    with torch.cuda.stream(stream):
+        med, mean, mn = _time_launches(lambda: gk.gkd_roi_to_image(xy, boxes_d, shape.B, shape.K, canvas, pts, stream),
+                                       stream, launches)
+    out["roi_to_image"] = {"launch_us": 1e6 * mean, "launch_us_median": 1e6 * med,
+                           "points_per_launch": shape.B * shape.K, "bound": "launch latency (B K points)"}
+    del img_d, boxes_d, canv, xy, pts
     gk.gkd_check_device_error(stream)
     return out
 

@@ -58,40 +58,57 @@ __device__ __forceinline__ AxisTap axis_tap(int d, int n_in, double origin, doub
   return t;
 }
 
+__device__ __forceinline__ float normalise(double v, int c) {
+  const double mean[3] = {0.485, 0.456, 0.406};
+  const double stdv[3] = {0.229, 0.224, 0.225};
+  return static_cast<float>(__ddiv_rn(__dsub_rn(__ddiv_rn(v, 255.0), mean[c]), stdv[c]));
+}
+
+// One CTA per (box, band of kPpRows canvas rows). Every value is computed as
+// the per-pixel formulas state; what depends on one axis only is computed once
+// and reused: the box geometry per thread, the row taps per band (shared
+// memory), a column's taps once for the band's rows, and the normalised pad
+// colour once per thread.
+constexpr int kPpRows = 8;
+
 __global__ void __launch_bounds__(256) preprocess_kernel(const uint8_t* __restrict__ img, int H, int W,
                                                          const float* __restrict__ boxes, int canvas,
                                                          float* __restrict__ out) {
+  __shared__ AxisTap rowtap[kPpRows];
   const int b = blockIdx.y;
+  const int Y0 = blockIdx.x * kPpRows;
+  const int nr = min(kPpRows, canvas - Y0);
   const long long npx = static_cast<long long>(canvas) * canvas;
-  const long long p = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (p >= npx) return;
-  const int Y = static_cast<int>(p / canvas), X = static_cast<int>(p % canvas);
   const BoxGeom g = box_geom(boxes + 4 * static_cast<long long>(b), canvas);
-  const double pad[3] = {124.0, 116.0, 104.0};
-  const double mean[3] = {0.485, 0.456, 0.406};
-  const double stdv[3] = {0.229, 0.224, 0.225};
-  double v[3] = {pad[0], pad[1], pad[2]};
-  if (g.ok) {
-    const AxisTap tx = axis_tap(X, W, g.x0, g.s, g.ox, g.bw);
-    const AxisTap ty = axis_tap(Y, H, g.y0, g.s, g.oy, g.bh);
-    if (tx.inside && ty.inside) {
-      const uint8_t* r0 = img + static_cast<long long>(ty.i0) * W * 3;
-      const uint8_t* r1 = img + static_cast<long long>(ty.i1) * W * 3;
-      const double wx0 = __dsub_rn(1.0, tx.lam), wy0 = __dsub_rn(1.0, ty.lam);
+  if (g.ok && threadIdx.x < nr) rowtap[threadIdx.x] = axis_tap(Y0 + threadIdx.x, H, g.y0, g.s, g.oy, g.bh);
+  __syncthreads();
+  const float padn[3] = {normalise(124.0, 0), normalise(116.0, 1), normalise(104.0, 2)};
+  float* ob = out + static_cast<long long>(b) * 3 * npx + static_cast<long long>(Y0) * canvas;
+  for (int X = threadIdx.x; X < canvas; X += blockDim.x) {
+    AxisTap tx{};
+    if (g.ok) tx = axis_tap(X, W, g.x0, g.s, g.ox, g.bw);
+    const double wx0 = __dsub_rn(1.0, tx.lam);
+    for (int r = 0; r < nr; ++r) {
+      float o[3] = {padn[0], padn[1], padn[2]};
+      if (g.ok && tx.inside && rowtap[r].inside) {
+        const AxisTap ty = rowtap[r];
+        const uint8_t* r0 = img + static_cast<long long>(ty.i0) * W * 3;
+        const uint8_t* r1 = img + static_cast<long long>(ty.i1) * W * 3;
+        const double wy0 = __dsub_rn(1.0, ty.lam);
 #pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        const double a = r0[3 * tx.i0 + c], bb = r0[3 * tx.i1 + c];
-        const double cc = r1[3 * tx.i0 + c], d = r1[3 * tx.i1 + c];
-        const double top = __dadd_rn(__dmul_rn(wx0, a), __dmul_rn(tx.lam, bb));
-        const double bot = __dadd_rn(__dmul_rn(wx0, cc), __dmul_rn(tx.lam, d));
-        v[c] = __dadd_rn(__dmul_rn(wy0, top), __dmul_rn(ty.lam, bot));
+        for (int c = 0; c < 3; ++c) {
+          const double a = r0[3 * tx.i0 + c], bb = r0[3 * tx.i1 + c];
+          const double cc = r1[3 * tx.i0 + c], d = r1[3 * tx.i1 + c];
+          const double top = __dadd_rn(__dmul_rn(wx0, a), __dmul_rn(tx.lam, bb));
+          const double bot = __dadd_rn(__dmul_rn(wx0, cc), __dmul_rn(tx.lam, d));
+          o[c] = normalise(__dadd_rn(__dmul_rn(wy0, top), __dmul_rn(ty.lam, bot)), c);
+        }
       }
+      const long long q = static_cast<long long>(r) * canvas + X;
+#pragma unroll
+      for (int c = 0; c < 3; ++c) ob[c * npx + q] = o[c];
     }
   }
-  float* ob = out + static_cast<long long>(b) * 3 * npx + p;
-#pragma unroll
-  for (int c = 0; c < 3; ++c)
-    ob[c * npx] = static_cast<float>(__ddiv_rn(__dsub_rn(__ddiv_rn(v[c], 255.0), mean[c]), stdv[c]));
 }
 
 __global__ void __launch_bounds__(256) roi_to_image_kernel(const float* __restrict__ xy,
@@ -115,8 +132,7 @@ __global__ void __launch_bounds__(256) roi_to_image_kernel(const float* __restri
 cudaError_t launch_preprocess(const uint8_t* img, int H, int W, const float* boxes, int B, int canvas, float* out,
                               cudaStream_t stream) {
   if (B == 0) return cudaSuccess;
-  const long long npx = static_cast<long long>(canvas) * canvas;
-  dim3 grid(static_cast<unsigned>((npx + 255) / 256), B);
+  dim3 grid(static_cast<unsigned>((canvas + kPpRows - 1) / kPpRows), B);
   preprocess_kernel<<<grid, 256, 0, stream>>>(img, H, W, boxes, canvas, out);
   return cudaGetLastError();
 }

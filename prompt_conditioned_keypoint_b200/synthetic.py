@@ -287,3 +287,17 @@ def random_heatmaps(seed: int, B: int, M: int, K: int, H: int, W: int, *, ties: 
             flat[r, g.integers(0, H * W)] = np.float32(0.0)
             flat[r, g.integers(0, H * W)] = np.float32(-0.0)
     return heat
+
+
+def random_image_and_boxes(seed: int, H: int, W: int, B: int) -> tuple[np.ndarray, np.ndarray]:
+    """A uint8 RGB frame [H][W][3] of uniform noise and B detector boxes
+    (x0, y0, x1, y1) fp32 inside it, each side 10-60% of the frame's, for the
+    preprocessing step and the ROI -> image map."""
+    g = _rng(seed, _FEAT, 123)
+    img = g.integers(0, 256, (H, W, 3), dtype=np.uint8)
+    bw = g.uniform(0.1, 0.6, B) * W
+    bh = g.uniform(0.1, 0.6, B) * H
+    x0 = g.uniform(0, 1, B) * (W - bw)
+    y0 = g.uniform(0, 1, B) * (H - bh)
+    boxes = np.stack([x0, y0, x0 + bw, y0 + bh], axis=1).astype(np.float32)
+    return img, boxes

@@ -61,3 +61,17 @@ def test_bf16_storage_cast_matches_torch():
                         np.array([0.0, -0.0, 1.00390625, 1.01171875, -1.00390625, 3.3e38, 1e-45], np.float32)])
     want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     np.testing.assert_array_equal(S.to_bf16_bits(x), want)
+
+
+def test_image_and_boxes_are_seeded_and_inside_the_frame():
+    from prompt_conditioned_keypoint_b200 import synthetic as S
+    img, boxes = S.random_image_and_boxes(7, 108, 192, 16)
+    img2, boxes2 = S.random_image_and_boxes(7, 108, 192, 16)
+    assert img.shape == (108, 192, 3) and img.dtype == np.uint8
+    assert boxes.shape == (16, 4) and boxes.dtype == np.float32
+    assert np.array_equal(img, img2) and np.array_equal(boxes, boxes2)
+    assert np.all(boxes[:, 0] >= 0) and np.all(boxes[:, 1] >= 0)
+    assert np.all(boxes[:, 2] <= 192 + 1e-3) and np.all(boxes[:, 3] <= 108 + 1e-3)
+    w, h = boxes[:, 2] - boxes[:, 0], boxes[:, 3] - boxes[:, 1]
+    assert np.all(w >= 0.1 * 192 - 1e-3) and np.all(w <= 0.6 * 192 + 1e-3)
+    assert np.all(h >= 0.1 * 108 - 1e-3) and np.all(h <= 0.6 * 108 + 1e-3)
